@@ -1,0 +1,180 @@
+"""CPU oracle for per-group INT4 RTN quantization and the W4A16 linear layer.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+CPU-baseline leg of the benchmark may import this package; the CUDA library
+never does, and the two share no code.  The arithmetic lives in ``w4ref.c``
+(plain scalar C, fp32 IEEE quantizer, fp64 dequantization and matmul); this
+module only builds it with gcc and marshals numpy arrays through ctypes.
+
+Sources followed (see ``w4ref.c`` for the step-by-step citations):
+"LLM quantization methods: principles and implementation"
+(zhiyuanblog.org/blog/llm-quantization) §2.2-§2.3 and §4.2, and
+"PTQ weight quantization: from GPTQ to AWQ" (jonathanding.github.io),
+sections "Round-to-Nearest" and "AWQ".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "w4ref.c")
+_LIB = os.path.join(_HERE, "libw4ref.so")
+
+F16 = 0
+BF16 = 1
+
+OK = 0
+EINVAL = 1
+ENONFINITE = 5
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile w4ref.c into libw4ref.so next to it (gcc, OpenMP, no FP contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
+               "-fPIC", "-shared", "-Wall", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        L = ctypes.c_long
+        I = ctypes.c_int
+        lib.w4ref_quantize.argtypes = [P, I, L, L, L, I, P, P, P, P]
+        lib.w4ref_quantize.restype = I
+        lib.w4ref_dequant.argtypes = [P, P, P, L, L, L, P]
+        lib.w4ref_dequant.restype = I
+        lib.w4ref_linear.argtypes = [P, I, L, L, P, L, P, L, P]
+        lib.w4ref_linear.restype = I
+        lib.w4ref_linear_at.argtypes = [P, I, L, P, P, P, L, L, L]
+        lib.w4ref_linear_at.restype = ctypes.c_double
+        lib.w4ref_code.argtypes = [P, L, L, L]
+        lib.w4ref_code.restype = I
+        lib.w4ref_f16_to_f64.argtypes = [ctypes.c_uint16]
+        lib.w4ref_f16_to_f64.restype = ctypes.c_double
+        lib.w4ref_bf16_to_f64.argtypes = [ctypes.c_uint16]
+        lib.w4ref_bf16_to_f64.restype = ctypes.c_double
+        lib.w4ref_threads.argtypes = []
+        lib.w4ref_threads.restype = I
+        lib.w4ref_set_threads.argtypes = [I]
+        lib.w4ref_set_threads.restype = None
+        _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else ctypes.c_void_p(a.ctypes.data)
+
+
+def _bits16(a: np.ndarray) -> np.ndarray:
+    """Accept uint16 bit patterns or np.float16 values; return contiguous uint16 bits."""
+    if a.dtype == np.float16:
+        a = a.view(np.uint16)
+    if a.dtype != np.uint16:
+        raise TypeError("16-bit inputs are passed as uint16 bit patterns or float16")
+    return np.ascontiguousarray(a)
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def set_threads(n: int) -> None:
+    _load().w4ref_set_threads(int(n))
+
+
+def threads() -> int:
+    return int(_load().w4ref_threads())
+
+
+def quantize(W, dtype: int, group: int, sym: bool, col_scale=None):
+    """Quantize W [N][K] -> (packed uint8 [N][K/2], scales f32 [N][G], zeros f32 [N][G])."""
+    W = _bits16(W)
+    N, K = W.shape
+    if col_scale is not None:
+        col_scale = np.ascontiguousarray(col_scale, dtype=np.float32)
+        assert col_scale.shape == (K,)
+    G = K // group if group > 0 else 0
+    packed = np.zeros((N, K // 2), np.uint8)
+    scales = np.zeros((N, max(G, 1)), np.float32)
+    zeros = np.zeros((N, max(G, 1)), np.float32)
+    st = _load().w4ref_quantize(_ptr(W), dtype, K, N, group, int(bool(sym)), _ptr(col_scale),
+                                _ptr(packed), _ptr(scales), _ptr(zeros))
+    if st != OK:
+        raise OracleError(f"w4ref_quantize status {st}")
+    return packed, scales[:, :G], zeros[:, :G]
+
+
+def dequant(packed, scales, zeros, K: int, group: int) -> np.ndarray:
+    """fp64 W-hat [N][K] = (u - zero) * scale; zeros=None means zero = 8 (symmetric)."""
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.float32)
+    if zeros is not None:
+        zeros = np.ascontiguousarray(zeros, dtype=np.float32)
+    N = packed.shape[0]
+    out = np.empty((N, K), np.float64)
+    st = _load().w4ref_dequant(_ptr(packed), _ptr(scales), _ptr(zeros), K, N, group, _ptr(out))
+    if st != OK:
+        raise OracleError(f"w4ref_dequant status {st}")
+    return out
+
+
+def linear(X, dtype: int, What: np.ndarray, rows=None) -> np.ndarray:
+    """fp64 Y = X * W-hat^T (naive loop); rows selects a subset of X's rows."""
+    X = _bits16(X)
+    M, K = X.shape
+    What = np.ascontiguousarray(What, dtype=np.float64)
+    N = What.shape[0]
+    assert What.shape[1] == K
+    if rows is not None:
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        nr = rows.shape[0]
+    else:
+        nr = M
+    Y = np.zeros((nr, N), np.float64)
+    st = _load().w4ref_linear(_ptr(X), dtype, M, K, _ptr(What), N, _ptr(rows), nr, _ptr(Y))
+    if st != OK:
+        raise OracleError(f"w4ref_linear status {st}")
+    return Y
+
+
+def linear_at(X, dtype: int, packed, scales, zeros, group: int, pairs) -> np.ndarray:
+    """fp64 Y[m][n] for a list of (m, n) pairs, straight from the packed weights."""
+    X = _bits16(X)
+    M, K = X.shape
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.float32)
+    if zeros is not None:
+        zeros = np.ascontiguousarray(zeros, dtype=np.float32)
+    lib = _load()
+    out = np.empty(len(pairs), np.float64)
+    for i, (m, n) in enumerate(pairs):
+        out[i] = lib.w4ref_linear_at(_ptr(X), dtype, K, _ptr(packed), _ptr(scales), _ptr(zeros),
+                                     group, int(m), int(n))
+    return out
+
+
+def code(packed, K: int, n: int, k: int) -> int:
+    """The 4-bit code of weight (n, k) read back from the packed layout."""
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    return int(_load().w4ref_code(_ptr(packed), K, n, k))
+
+
+def f16_to_f64(h: int) -> float:
+    return float(_load().w4ref_f16_to_f64(h))
+
+
+def bf16_to_f64(h: int) -> float:
+    return float(_load().w4ref_bf16_to_f64(h))

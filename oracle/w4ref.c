@@ -1,0 +1,293 @@
+/*
+ * w4ref.c -- CPU oracle for per-group INT4 round-to-nearest weight quantization
+ * and the W4A16 linear layer.  TEST INFRASTRUCTURE ONLY: only the test suite,
+ * the smoke check and the CPU-baseline leg of the benchmark may load it.  It
+ * shares no code, header, table or helper with the CUDA library and it is
+ * never part of the product path.
+ *
+ * Plain, slow, scalar C.  Every step follows the method as the source pages
+ * state it, in their order:
+ *
+ *   [LQ]  "LLM quantization methods: principles and implementation"
+ *         (zhiyuanblog.org/blog/llm-quantization)
+ *         §2.2 integer quantization maths: symmetric  s = max|x| / (2^(b-1)-1),
+ *              x_q = clamp(round(x/s), -qmax, qmax), x ~ x_q * s;
+ *              asymmetric s = (max-min)/(2^b-1), zero_point = clamp(round(-min/s), 0, 2^b-1),
+ *              x_q = clamp(round(x/s + zero_point), 0, 2^b-1), x ~ (x_q - zero_point) * s.
+ *         §2.3 per-group granularity: W is (out_features, in_features), the in
+ *              dimension is cut into groups of g (e.g. 128) with one scale each,
+ *              and in_features must be a multiple of g.
+ *         §4.2 AWQ: W is multiplied column-wise by a per-input-channel factor s
+ *              before the per-group quantizer runs.
+ *   [PTQ] "PTQ weight quantization: from GPTQ to AWQ" (jonathanding.github.io),
+ *         section "Round-to-Nearest": every weight is rounded on its own to the
+ *         nearest level; section "AWQ": XW = (X diag(s)^-1)(diag(s) W).
+ *   [MF]  "Quantization method families" (inference-learning-path.pages.dev),
+ *         §2 mental model: W4A16 keeps activations in 16-bit floats and
+ *         dequantizes the weights before the matmul.
+ *
+ * Readings where the pages leave a step open (each one is also listed in the
+ * design notes of the repository):
+ *   - all scale / zero-point / division arithmetic is IEEE fp32 with
+ *     round-to-nearest-even; "round" is round-half-to-even (torch.round);
+ *   - the asymmetric path uses the code form of §2.2 (integer zero point),
+ *     rounding after the fp32 add: u = rne(fl(fl(w/s) + zp));
+ *   - symmetric codes q in [-7, 7] are stored as u = q + 8 with zero = 8.0f,
+ *     so both forms dequantize as (u - zero) * scale;
+ *   - a group whose scale comes out 0 (all-zero symmetric group, constant
+ *     asymmetric group) stores scale 0, zero 8 (sym) or 0 (asym) and u = zero,
+ *     so it dequantizes to 0;
+ *   - nibble layout (ours; the pages give only "0.5 byte per parameter"):
+ *     packed is [N][K/2] bytes; the 8 codes of k = 8j..8j+7 of a row form the
+ *     little-endian 32-bit word j, whose nibble i (bits 4i..4i+3) holds
+ *     k = 8j + SIGMA[i] with SIGMA = {0,2,4,6,1,3,5,7};
+ *   - scales and zeros are fp32 [N][K/group].
+ *
+ * Compiled with -O2 -ffp-contract=off -fno-fast-math so that every float
+ * operation below is one correctly rounded IEEE binary32 operation.
+ */
+#include <fenv.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#define W4REF_OK 0
+#define W4REF_EINVAL 1
+#define W4REF_ENONFINITE 5
+
+#define DT_F16 0
+#define DT_BF16 1
+
+/* Position of k-within-word for nibble i of a packed 32-bit word. */
+static const int SIGMA[8] = {0, 2, 4, 6, 1, 3, 5, 7};
+
+/* ---- 16-bit float decoding, from the IEEE 754 binary16 and bfloat16 definitions ---- */
+
+/* binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits. */
+double w4ref_f16_to_f64(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1F;
+    int f = h & 0x3FF;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -24); /* subnormal: f * 2^-24 */
+    else if (e == 31)
+        v = f ? NAN : INFINITY;
+    else
+        v = ldexp((double)(1024 + f), e - 25); /* (1 + f/1024) * 2^(e-15) */
+    return sign ? -v : v;
+}
+
+/* bfloat16 is the upper half of an IEEE binary32. */
+double w4ref_bf16_to_f64(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static double decode16(uint16_t h, int dtype)
+{
+    return dtype == DT_BF16 ? w4ref_bf16_to_f64(h) : w4ref_f16_to_f64(h);
+}
+
+/* Round-to-nearest, ties to even (torch.round), in the current FE_TONEAREST mode. */
+static float rne(float x) { return nearbyintf(x); }
+
+static float clampf(float v, float lo, float hi)
+{
+    if (v < lo) return lo;
+    if (v > hi) return hi;
+    return v;
+}
+
+/* ---- quantize ------------------------------------------------------------------ */
+
+/*
+ * Quantize W [N][K] (fp16 or bf16 bit patterns, row-major, out x in) group by
+ * group along K.  col_scale (nullable, [K] fp32) is the AWQ per-input-channel
+ * factor folded in first: w = fl32(w * col_scale[k]).
+ * Outputs: packed [N][K/2], scales [N][K/group], zeros [N][K/group].
+ * group must divide K, be a multiple of 8 and be at most 4096.
+ * Returns W4REF_EINVAL on a bad shape, W4REF_ENONFINITE if a folded weight,
+ * a group range or a scale is not finite (that group's outputs are not written).
+ */
+int w4ref_quantize(const uint16_t *W, int dtype, long K, long N, long group, int sym,
+                   const float *col_scale, uint8_t *packed, float *scales, float *zeros)
+{
+    if (K <= 0 || N <= 0 || group <= 0 || group > 4096 || group % 8 != 0 || K % group != 0)
+        return W4REF_EINVAL;
+    if (dtype != DT_F16 && dtype != DT_BF16) return W4REF_EINVAL;
+    fesetround(FE_TONEAREST);
+    const long G = K / group;
+    int status = W4REF_OK;
+
+#pragma omp parallel for schedule(static)
+    for (long n = 0; n < N; ++n) {
+        float w[4096];
+        uint8_t u[4096];
+        for (long g = 0; g < G; ++g) {
+            const long k0 = g * group;
+            /* step 1: load, optional AWQ fold (one fp32 multiply) */
+            int bad = 0;
+            for (long i = 0; i < group; ++i) {
+                float v = (float)decode16(W[n * K + k0 + i], dtype);
+                if (col_scale) v = v * col_scale[k0 + i];
+                if (!isfinite(v)) bad = 1;
+                w[i] = v;
+            }
+            float s, z;
+            if (sym) {
+                /* step 2: amax = max |w|; step 3: s = amax / qmax, qmax = 2^(4-1)-1 = 7 */
+                float amax = 0.0f;
+                for (long i = 0; i < group; ++i) {
+                    float a = fabsf(w[i]);
+                    if (a > amax) amax = a;
+                }
+                s = amax / 7.0f;
+                z = 8.0f;
+                if (!isfinite(s)) bad = 1;
+                if (!bad) {
+                    for (long i = 0; i < group; ++i) {
+                        if (s == 0.0f) { u[i] = 8; continue; }
+                        /* step 4: q = clamp(round(w / s), -7, 7); stored as q + 8 */
+                        float q = clampf(rne(w[i] / s), -7.0f, 7.0f);
+                        u[i] = (uint8_t)((int)q + 8);
+                    }
+                }
+            } else {
+                /* step 2: min and max of the group; step 3: s = (max - min) / (2^4 - 1) */
+                float mn = w[0], mx = w[0];
+                for (long i = 1; i < group; ++i) {
+                    if (w[i] < mn) mn = w[i];
+                    if (w[i] > mx) mx = w[i];
+                }
+                float range = mx - mn;
+                s = range / 15.0f;
+                if (!isfinite(range) || !isfinite(s)) bad = 1;
+                if (!bad) {
+                    if (s == 0.0f) {
+                        z = 0.0f;
+                        for (long i = 0; i < group; ++i) u[i] = 0;
+                    } else {
+                        /* zero_point = clamp(round(-min / s), 0, 15) */
+                        float negmn = -mn;
+                        z = clampf(rne(negmn / s), 0.0f, 15.0f);
+                        for (long i = 0; i < group; ++i) {
+                            /* step 4: u = clamp(round(w / s + zero_point), 0, 15) */
+                            float t = w[i] / s;
+                            float y = t + z;
+                            float q = clampf(rne(y), 0.0f, 15.0f);
+                            u[i] = (uint8_t)(int)q;
+                        }
+                    }
+                } else {
+                    z = 0.0f;
+                }
+            }
+            if (bad) {
+#pragma omp atomic write
+                status = W4REF_ENONFINITE;
+                continue;
+            }
+            scales[n * G + g] = s;
+            zeros[n * G + g] = z;
+            /* step 5: pack 8 codes per 32-bit little-endian word */
+            for (long j = 0; j < group / 8; ++j) {
+                uint32_t word = 0;
+                for (int i = 0; i < 8; ++i) word |= (uint32_t)(u[j * 8 + SIGMA[i]] & 0xF) << (4 * i);
+                uint8_t *dst = packed + n * (K / 2) + (k0 + j * 8) / 2;
+                for (int b = 0; b < 4; ++b) dst[b] = (uint8_t)(word >> (8 * b));
+            }
+        }
+    }
+    return status;
+}
+
+/* ---- unpack / dequantize ----------------------------------------------------------- */
+
+/* Code u of (n, k) from packed [N][K/2]: the inverse of the packing above. */
+int w4ref_code(const uint8_t *packed, long K, long n, long k)
+{
+    long j = k / 8, r = k % 8;
+    const uint8_t *src = packed + n * (K / 2) + j * 4;
+    uint32_t word = (uint32_t)src[0] | ((uint32_t)src[1] << 8) | ((uint32_t)src[2] << 16) |
+                    ((uint32_t)src[3] << 24);
+    for (int i = 0; i < 8; ++i)
+        if (SIGMA[i] == r) return (int)((word >> (4 * i)) & 0xF);
+    return -1;
+}
+
+/*
+ * What [N][K] (fp64) = (u - zero) * scale, computed exactly in fp64.
+ * zeros == NULL means the symmetric storage (zero = 8).
+ */
+int w4ref_dequant(const uint8_t *packed, const float *scales, const float *zeros, long K,
+                  long N, long group, double *What)
+{
+    if (K <= 0 || N <= 0 || group <= 0 || K % group != 0 || K % 8 != 0) return W4REF_EINVAL;
+    const long G = K / group;
+#pragma omp parallel for schedule(static)
+    for (long n = 0; n < N; ++n)
+        for (long k = 0; k < K; ++k) {
+            double s = (double)scales[n * G + k / group];
+            double z = zeros ? (double)zeros[n * G + k / group] : 8.0;
+            What[n * K + k] = ((double)w4ref_code(packed, K, n, k) - z) * s;
+        }
+    return W4REF_OK;
+}
+
+/* ---- the W4A16 linear layer ------------------------------------------------------------ */
+
+/*
+ * Y[m][n] = sum_k X[m][k] * What[n][k], naive fp64 loop in k order.
+ * X [M][K] holds fp16/bf16 bit patterns.  rows (nullable) selects the m to
+ * compute; Y is then [nrows][N] in the order of rows.
+ */
+int w4ref_linear(const uint16_t *X, int dtype, long M, long K, const double *What, long N,
+                 const long *rows, long nrows, double *Y)
+{
+    if (M <= 0 || K <= 0 || N <= 0) return W4REF_EINVAL;
+    if (!rows) nrows = M;
+#pragma omp parallel for schedule(static)
+    for (long r = 0; r < nrows; ++r) {
+        long m = rows ? rows[r] : r;
+        if (m < 0 || m >= M) continue;
+        for (long n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (long k = 0; k < K; ++k) acc += decode16(X[m * K + k], dtype) * What[n * K + k];
+            Y[r * N + n] = acc;
+        }
+    }
+    return W4REF_OK;
+}
+
+/*
+ * Same product straight from the packed weights, for one (m, n) pair at a
+ * time: used where the full fp64 W-hat would not fit (sampled checks).
+ */
+double w4ref_linear_at(const uint16_t *X, int dtype, long K, const uint8_t *packed,
+                       const float *scales, const float *zeros, long group, long m, long n)
+{
+    const long G = K / group;
+    double acc = 0.0;
+    for (long k = 0; k < K; ++k) {
+        double s = (double)scales[n * G + k / group];
+        double z = zeros ? (double)zeros[n * G + k / group] : 8.0;
+        double w = ((double)w4ref_code(packed, K, n, k) - z) * s;
+        acc += decode16(X[m * K + k], dtype) * w;
+    }
+    return acc;
+}
+
+/* Number of OpenMP threads the parallel loops above use (1 without OpenMP). */
+#ifdef _OPENMP
+#include <omp.h>
+int w4ref_threads(void) { return omp_get_max_threads(); }
+void w4ref_set_threads(int n) { omp_set_num_threads(n); }
+#else
+int w4ref_threads(void) { return 1; }
+void w4ref_set_threads(int n) { (void)n; }
+#endif
