@@ -1,0 +1,139 @@
+/*
+ * w4a16.h -- C ABI of libw4a16.so: per-group INT4 round-to-nearest weight
+ * quantization and the W4A16 linear layer on NVIDIA B200 (sm_100a).
+ *
+ * Method sources (cited by page title and section):
+ *   [LQ]  "LLM quantization methods: principles and implementation"
+ *         (zhiyuanblog.org/blog/llm-quantization): §1 (0.5 byte per INT4
+ *         parameter), §2.2 (symmetric and asymmetric integer quantization,
+ *         scale and zero point, round, clamp, dequantize), §2.3 (per-group
+ *         granularity along in_features, in_features % group == 0),
+ *         §4.2 (AWQ: weights multiplied by a per-input-channel factor before
+ *         quantizing).
+ *   [PTQ] "PTQ weight quantization: from GPTQ to AWQ" (jonathanding.github.io),
+ *         sections "Round-to-Nearest" and "AWQ".
+ *   [MF]  "Quantization method families" (inference-learning-path.pages.dev),
+ *         §2: W4A16 keeps activations in 16-bit floats and dequantizes the
+ *         weights in front of the matmul; decode is bound by weight bandwidth,
+ *         prefill by compute.
+ *
+ * Conventions shared by every entry point:
+ *   - All array arguments are DEVICE pointers of the current CUDA device,
+ *     allocated and owned by the caller; the library allocates no memory.
+ *     Base pointers must be 16-byte aligned (else W4_ERR_UNSUPPORTED).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Every call only enqueues work and returns: results are ready once the
+ *     caller synchronizes that stream.  Launch failures return W4_ERR_CUDA;
+ *     faults inside a kernel surface at the caller's synchronization.
+ *   - Arguments are validated on the host before anything is enqueued; an
+ *     invalid call returns its status and touches no memory.
+ *   - Matrices are row-major.  W is [N][K] = (out_features x in_features); X is
+ *     [M][K]; Y is [M][N].  Groups run along K (in_features).
+ *   - Inputs must be finite; results for NaN or Inf inputs are unspecified.
+ *   - Thread safety: calls on different streams may run concurrently; the
+ *     library keeps no per-call host state beyond a per-device cache of
+ *     attributes (SM count, kernel attributes) filled on first use.
+ */
+#ifndef W4A16_H
+#define W4A16_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    W4_OK = 0,
+    W4_ERR_INVALID_ARG = 1, /* bad shape, null pointer, K % group != 0, ... */
+    W4_ERR_UNSUPPORTED = 2, /* valid but not implemented (group size, alignment, dtype) */
+    W4_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed while enqueueing */
+    W4_ERR_TIMEOUT = 4      /* a bounded device-side wait ran out (see w4_device_status) */
+} w4_status;
+
+typedef enum { W4_F16 = 0, W4_BF16 = 1 } w4_dtype;
+
+/*
+ * w4_quantize -- per-group INT4 round-to-nearest quantization and packing.
+ * [LQ] §2.2 + §2.3 (+ §4.2 for col_scale); [PTQ] "Round-to-Nearest".
+ *
+ *   W          [N][K] fp16 or bf16 (wt), the weight (out x in).
+ *   col_scale  nullable [K] fp32: AWQ per-input-channel factor; when given,
+ *              every weight is first replaced by fl32(w * col_scale[k]).
+ *   group      elements per group along K: 32, 64, 128 or 256; K % group == 0
+ *              (W4_ERR_INVALID_ARG otherwise).
+ *   sym != 0   symmetric:  s = fl(amax / 7), q = clamp(rne(fl(w / s)), -7, 7),
+ *              stored code u = q + 8, zeros[] = 8.0f.
+ *   sym == 0   asymmetric: s = fl(fl(max - min) / 15),
+ *              zp = clamp(rne(fl(-min / s)), 0, 15),
+ *              u = clamp(rne(fl(fl(w / s) + zp)), 0, 15), zeros[] = zp.
+ *   All arithmetic is IEEE fp32 with round-to-nearest-even; rne() rounds
+ *   half to even.  A group whose scale is 0 stores s = 0, zero = 8 (sym) or
+ *   0 (asym) and every code equal to that zero, so it dequantizes to 0.
+ *   Outputs (caller-allocated):
+ *     packed   [N][K/2] bytes.  The codes of k = 8j..8j+7 of a row form the
+ *              little-endian 32-bit word j; nibble i (bits 4i..4i+3) of that
+ *              word holds k = 8j + {0,2,4,6,1,3,5,7}[i].
+ *     scales   [N][K/group] fp32.
+ *     zeros    [N][K/group] fp32 (integer values 0..15).
+ *   Dequantization of any code: w_hat = (u - zero) * scale.
+ *   Requires K % 8 == 0, N >= 1, K >= 1.
+ */
+int w4_quantize(const void *W, int wt, int64_t K, int64_t N, int group, int sym,
+                const float *col_scale, uint8_t *packed, float *scales, float *zeros,
+                void *stream);
+
+/*
+ * w4a16_workspace_bytes -- scratch bytes w4a16_gemm needs for this shape
+ * (0 when it needs none).  The workspace holds split-K partial sums and
+ * per-tile arrival counters; it must be zero-filled once before its first
+ * use, and w4a16_gemm leaves it zero-filled again when its work completes,
+ * so one workspace can serve any number of calls issued on ONE stream
+ * (calls that may overlap need separate workspaces).
+ */
+size_t w4a16_workspace_bytes(int64_t M, int64_t K, int64_t N, int group);
+
+/*
+ * w4a16_gemm -- Y = X * dequant(packed, scales, zeros)^T, the W4A16 linear layer.
+ * [MF] §2 (dequant -> 16-bit matmul); dequantization as in [LQ] §2.2.
+ *
+ *   X        [M][K] fp16 or bf16 (xt); Y [M][N] in the same dtype.
+ *   packed, scales, zeros: the layout w4_quantize writes; zeros may be NULL,
+ *            which means every zero point is 8 (the symmetric storage).
+ *   group    must be 128 (W4_ERR_UNSUPPORTED otherwise).
+ *   Each Y[m][n] = sum_k X[m][k] * ((u[n][k] - zero) * scale) is accumulated in
+ *   fp32 (the integer (u - zero) is exact in the 16-bit operand type; the
+ *   group scale multiplies the fp32 partial sum of its group) and rounded
+ *   once to the output dtype.
+ *   M <= 32 runs the decode path (split-K tensor-core GEMV); larger M runs
+ *   the tcgen05 path (TMA-staged X, dequantized W tiles in shared memory,
+ *   accumulators in tensor memory).
+ *   workspace / workspace_bytes: at least w4a16_workspace_bytes(M, K, N, group)
+ *   bytes of device memory prepared as described there (may be NULL when
+ *   that size is 0); a smaller workspace returns W4_ERR_INVALID_ARG.
+ */
+int w4a16_gemm(const void *X, int xt, int64_t M, const uint8_t *packed, const float *scales,
+               const float *zeros, int64_t K, int64_t N, int group, void *Y, void *workspace,
+               size_t workspace_bytes, void *stream);
+
+/*
+ * w4_device_status -- reads (and, if reset != 0, clears) the current device's
+ * status word that kernels set when a bounded wait runs out.  Synchronizes the
+ * device first.  Returns W4_OK, W4_ERR_TIMEOUT, or W4_ERR_CUDA if the read fails.
+ */
+int w4_device_status(int reset);
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char *w4_status_string(int status);
+
+/* ABI version of this header: (major << 16) | minor. */
+int w4_abi_version(void);
+
+#define W4A16_ABI_VERSION 0x00010000
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A16_H */

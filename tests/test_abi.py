@@ -1,0 +1,123 @@
+"""The C ABI of libw4a16.so, checked without a GPU: it builds, loads, exports
+every function include/w4a16.h declares, and rejects invalid arguments with
+the documented status before anything reaches the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import weight_only_int4_pack_b200 as w4
+from weight_only_int4_pack_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return w4.load()
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if not fn.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", fn)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        for m in re.finditer(r"^\s*[A-Za-z_][\w\s\*]*?\b(w4\w*)\s*\(", src, flags=re.M):
+            names.append(m.group(1))
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ("w4_quantize", "w4a16_gemm", "w4a16_workspace_bytes", "w4_status_string",
+                 "w4_device_status", "w4_abi_version"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_abi_version_and_status_strings(lib):
+    assert w4.w4_abi_version() == 0x00010000
+    assert w4.w4_status_string(0) == "W4_OK"
+    assert w4.w4_status_string(1) == "W4_ERR_INVALID_ARG"
+    assert w4.w4_status_string(2) == "W4_ERR_UNSUPPORTED"
+    assert w4.w4_status_string(3) == "W4_ERR_CUDA"
+    assert w4.w4_status_string(4) == "W4_ERR_TIMEOUT"
+    assert w4.w4_status_string(99) == "W4_ERR_UNKNOWN"
+
+
+# Fake, 16-byte aligned, never-dereferenced addresses: validation must reject
+# before any of them is touched.
+A = ctypes.c_void_p(0x100000)
+B = ctypes.c_void_p(0x200000)
+C = ctypes.c_void_p(0x300000)
+D = ctypes.c_void_p(0x400000)
+S = ctypes.c_void_p(0)
+
+
+@pytest.mark.parametrize("args,status", [
+    # (W, wt, K, N, group, sym, col_scale, packed, scales, zeros)
+    ((A, 0, 192, 4, 128, 1, None, B, C, D), 1),    # K % group != 0 (the pages' assert)
+    ((A, 0, 0, 4, 128, 1, None, B, C, D), 1),      # K == 0
+    ((A, 0, 256, -1, 128, 1, None, B, C, D), 1),   # N < 0
+    ((A, 2, 256, 4, 128, 1, None, B, C, D), 1),    # bad dtype
+    ((A, 0, 256, 4, 0, 1, None, B, C, D), 1),      # group 0
+    ((None, 0, 256, 4, 128, 1, None, B, C, D), 1), # null W
+    ((A, 0, 256, 4, 128, 1, None, None, C, D), 1), # null packed
+    ((A, 0, 256, 4, 128, 1, None, B, None, D), 1), # null scales
+    ((A, 0, 256, 4, 128, 1, None, B, C, None), 1), # null zeros
+    ((A, 0, 132, 4, 4, 1, None, B, C, D), 1),      # K % 8 != 0
+    ((A, 0, 384, 4, 96, 1, None, B, C, D), 2),     # group not in {32,64,128,256}
+    ((A, 0, 512, 4, 512, 1, None, B, C, D), 2),
+    ((ctypes.c_void_p(0x100008), 0, 256, 4, 128, 1, None, B, C, D), 2),  # misaligned W
+    ((A, 0, 256, 4, 128, 1, ctypes.c_void_p(0x500004), B, C, D), 2),     # misaligned col_scale
+    ((A, 0, 256, 0, 128, 1, None, None, None, None), 0),  # N == 0: nothing to do
+])
+def test_quantize_argument_checks(lib, args, status):
+    assert lib.w4_quantize(*args, S) == status
+
+
+@pytest.mark.parametrize("args,status", [
+    # (X, xt, M, packed, scales, zeros, K, N, group, Y, ws, ws_bytes)
+    ((A, 0, 1, B, C, None, 192, 8, 128, D, None, 0), 1),   # K % group
+    ((A, 0, -1, B, C, None, 256, 8, 128, D, None, 0), 1),   # M < 0
+    ((A, 0, 1, B, C, None, 256, -3, 128, D, None, 0), 1),   # N < 0
+    ((A, 0, 1, B, C, None, 0, 8, 128, D, None, 0), 1),      # K == 0
+    ((A, 5, 1, B, C, None, 256, 8, 128, D, None, 0), 1),    # dtype
+    ((None, 0, 1, B, C, None, 256, 8, 128, D, None, 0), 1), # null X
+    ((A, 0, 1, None, C, None, 256, 8, 128, D, None, 0), 1), # null packed
+    ((A, 0, 1, B, None, None, 256, 8, 128, D, None, 0), 1), # null scales
+    ((A, 0, 1, B, C, None, 256, 8, 128, None, None, 0), 1), # null Y
+    ((A, 0, 1, B, C, None, 256, 8, 64, D, None, 0), 2),     # only group 128 multiplies
+    ((A, 0, 1, ctypes.c_void_p(0x200004), C, None, 256, 8, 128, D, None, 0), 2),  # misaligned
+    ((A, 0, 0, B, C, None, 256, 8, 128, D, None, 0), 0),    # M == 0: nothing to do
+    ((A, 0, 4, B, C, None, 256, 0, 128, D, None, 0), 0),    # N == 0: nothing to do
+])
+def test_gemm_argument_checks(lib, args, status):
+    assert lib.w4a16_gemm(*args, S) == status
+
+
+def test_product_path_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(w4, "lib_path", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(w4, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        w4.load()
+
+
+def test_product_package_does_not_reach_the_oracle():
+    pkg = os.path.join(ROOT, "weight_only_int4_pack_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if not fn.endswith((".py", ".cu", ".cuh", ".h")):
+                continue
+            src = open(os.path.join(dirpath, fn)).read()
+            assert "import oracle" not in src and "from oracle" not in src, fn
+            assert "w4ref" not in src and "libw4ref" not in src, fn

@@ -1,0 +1,187 @@
+"""Python binding of libw4a16.so: per-group INT4 weight quantization and the
+W4A16 linear layer on B200 (sm_100a).
+
+Argument marshalling only.  Every computation runs in the CUDA kernels of
+libw4a16.so; there is no Python or CPU fallback, and every call raises if the
+library is missing or returns an error status.  PyTorch provides device
+memory and streams.
+
+The functions mirror the C ABI of include/w4a16.h, with tensors in place of
+pointers:
+
+    w4_quantize(W, group=128, sym=True, col_scale=None) -> (packed, scales, zeros)
+    w4a16_workspace_bytes(M, K, N, group=128) -> int
+    w4a16_gemm(X, packed, scales, zeros, group=128, out=None, workspace=None) -> Y
+    w4_status_string(status) -> str
+    w4_device_status(reset=True) -> int
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "W4Error", "load", "lib_path", "w4_quantize", "w4_quantize_into", "w4a16_workspace_bytes",
+    "w4a16_gemm", "w4a16_gemm_into", "w4_status_string", "w4_device_status", "w4_abi_version",
+    "Workspace", "W4_OK", "W4_ERR_INVALID_ARG", "W4_ERR_UNSUPPORTED", "W4_ERR_CUDA",
+    "W4_ERR_TIMEOUT", "W4_F16", "W4_BF16",
+]
+
+W4_OK, W4_ERR_INVALID_ARG, W4_ERR_UNSUPPORTED, W4_ERR_CUDA, W4_ERR_TIMEOUT = 0, 1, 2, 3, 4
+W4_F16, W4_BF16 = 0, 1
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_PKG, "lib", "libw4a16.so")
+_lib = None
+
+
+class W4Error(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {w4_status_string(status)} ({status})")
+
+
+def load() -> ctypes.CDLL:
+    """Load libw4a16.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(lib_path):
+        raise RuntimeError(
+            f"{lib_path} is missing: build it with `python -m weight_only_int4_pack_b200.build`")
+    lib = ctypes.CDLL(lib_path)
+    P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    lib.w4_quantize.argtypes = [P, I, I64, I64, I, I, P, P, P, P, P]
+    lib.w4_quantize.restype = I
+    lib.w4a16_workspace_bytes.argtypes = [I64, I64, I64, I]
+    lib.w4a16_workspace_bytes.restype = SZ
+    lib.w4a16_gemm.argtypes = [P, I, I64, P, P, P, I64, I64, I, P, P, SZ, P]
+    lib.w4a16_gemm.restype = I
+    lib.w4_device_status.argtypes = [I]
+    lib.w4_device_status.restype = I
+    lib.w4_status_string.argtypes = [I]
+    lib.w4_status_string.restype = ctypes.c_char_p
+    lib.w4_abi_version.argtypes = []
+    lib.w4_abi_version.restype = I
+    _lib = lib
+    return lib
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float16:
+        return W4_F16
+    if t.dtype == torch.bfloat16:
+        return W4_BF16
+    raise TypeError(f"expected float16 or bfloat16, got {t.dtype}")
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_dev(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("tensors must live on a CUDA device")
+            if not t.is_contiguous():
+                raise ValueError("tensors must be contiguous")
+
+
+def w4_status_string(status: int) -> str:
+    try:
+        return load().w4_status_string(int(status)).decode()
+    except RuntimeError:
+        return str(status)
+
+
+def w4_abi_version() -> int:
+    return int(load().w4_abi_version())
+
+
+def w4_device_status(reset: bool = True) -> int:
+    """Status word set by kernels whose bounded waits ran out (synchronizes)."""
+    return int(load().w4_device_status(int(bool(reset))))
+
+
+def w4_quantize_into(W, packed, scales, zeros, group=128, sym=True, col_scale=None, stream=None):
+    """Quantize W [N][K] into caller-provided packed [N][K/2] u8, scales/zeros [N][K/group] f32."""
+    _check_dev(W, packed, scales, zeros, col_scale)
+    N, K = W.shape
+    st = load().w4_quantize(_p(W), _dt(W), K, N, int(group), int(bool(sym)), _p(col_scale),
+                            _p(packed), _p(scales), _p(zeros), _stream(stream))
+    if st != W4_OK:
+        raise W4Error("w4_quantize", st)
+    return packed, scales, zeros
+
+
+def w4_quantize(W: torch.Tensor, group: int = 128, sym: bool = True, col_scale=None, stream=None):
+    """Per-group INT4 RTN quantization of W [N][K] -> (packed, scales, zeros)."""
+    N, K = W.shape
+    G = K // group if group > 0 else 0
+    packed = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+    scales = torch.empty((N, G), dtype=torch.float32, device=W.device)
+    zeros = torch.empty((N, G), dtype=torch.float32, device=W.device)
+    return w4_quantize_into(W, packed, scales, zeros, group, sym, col_scale, stream)
+
+
+def w4a16_workspace_bytes(M: int, K: int, N: int, group: int = 128) -> int:
+    return int(load().w4a16_workspace_bytes(int(M), int(K), int(N), int(group)))
+
+
+class Workspace:
+    """A zero-filled device workspace that grows on demand (one per stream)."""
+
+    def __init__(self, device=None):
+        self.buf = None
+        self.device = device
+
+    def get(self, nbytes: int, device):
+        if nbytes == 0:
+            return None
+        if self.buf is None or self.buf.numel() < nbytes or self.buf.device != device:
+            self.buf = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
+        return self.buf
+
+
+_default_ws = {}
+
+
+def w4a16_gemm_into(X, packed, scales, zeros, Y, group=128, workspace=None, stream=None):
+    """Y [M][N] = X [M][K] * dequant(packed, scales, zeros)^T into caller-provided Y."""
+    _check_dev(X, packed, scales, zeros, Y)
+    M, K = X.shape
+    N = packed.shape[0]
+    lib = load()
+    need = int(lib.w4a16_workspace_bytes(M, K, N, int(group)))
+    if isinstance(workspace, Workspace) or workspace is None:
+        wsobj = workspace
+        if wsobj is None:
+            key = (X.device, (stream or torch.cuda.current_stream()).cuda_stream)
+            wsobj = _default_ws.setdefault(key, Workspace())
+        ws = wsobj.get(need, X.device)
+    else:
+        ws = workspace
+    wsz = 0 if ws is None else ws.numel() * ws.element_size()
+    st = lib.w4a16_gemm(_p(X), _dt(X), M, _p(packed), _p(scales), _p(zeros), K, N, int(group),
+                        _p(Y), _p(ws), wsz, _stream(stream))
+    if st != W4_OK:
+        raise W4Error("w4a16_gemm", st)
+    return Y
+
+
+def w4a16_gemm(X, packed, scales, zeros=None, group: int = 128, out=None, workspace=None,
+               stream=None):
+    """The W4A16 linear layer: Y = X * dequant(packed, scales, zeros)^T."""
+    M = X.shape[0]
+    N = packed.shape[0]
+    Y = out if out is not None else torch.empty((M, N), dtype=X.dtype, device=X.device)
+    return w4a16_gemm_into(X, packed, scales, zeros, Y, group, workspace, stream)

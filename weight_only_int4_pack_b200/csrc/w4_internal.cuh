@@ -1,0 +1,45 @@
+// w4_internal.cuh -- declarations shared by the CUDA translation units of
+// libw4a16.so.  Host-side launchers return w4_status codes; nothing here is
+// part of the public ABI (that is include/w4a16.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "w4a16.h"
+
+namespace w4 {
+
+// Per-device attributes cached on first use.
+struct DeviceInfo {
+    int sm_count = 0;
+    int cc_major = 0, cc_minor = 0;
+    int max_smem_optin = 0;
+    size_t l2_bytes = 0;
+};
+int device_info(DeviceInfo *out);  // W4_OK or W4_ERR_CUDA
+
+// Device address of the library's status word for the current device
+// (kernels set W4_ERR_TIMEOUT into it when a bounded wait runs out).
+unsigned *device_status_ptr();
+
+inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? W4_OK : W4_ERR_CUDA; }
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---- launchers (one per translation unit) ----
+int launch_quantize(const void *W, int wt, int64_t K, int64_t N, int group, int sym,
+                    const float *col_scale, uint8_t *packed, float *scales, float *zeros,
+                    cudaStream_t stream);
+
+// decode path, M <= 32
+size_t decode_workspace_bytes(int64_t M, int64_t K, int64_t N, int group);
+int launch_decode(const void *X, int xt, int64_t M, const uint8_t *packed, const float *scales,
+                  const float *zeros, int64_t K, int64_t N, void *Y, void *workspace,
+                  size_t workspace_bytes, cudaStream_t stream);
+
+// prefill path, M > 32 (tcgen05)
+int launch_prefill(const void *X, int xt, int64_t M, const uint8_t *packed, const float *scales,
+                   const float *zeros, int64_t K, int64_t N, void *Y, cudaStream_t stream);
+
+}  // namespace w4
