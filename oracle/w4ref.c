@@ -175,6 +175,8 @@ int w4ref_quantize(const uint16_t *W, int dtype, long K, long N, long group, int
                         /* zero_point = clamp(round(-min / s), 0, 15) */
                         float negmn = -mn;
                         z = clampf(rne(negmn / s), 0.0f, 15.0f);
+                        /* the zero point is an integer in [0, 15]; store 0 as +0.0 */
+                        z = z + 0.0f;
                         for (long i = 0; i < group; ++i) {
                             /* step 4: u = clamp(round(w / s + zero_point), 0, 15) */
                             float t = w[i] / s;
