@@ -86,11 +86,13 @@ int w4_quantize(const void *W, int wt, int64_t K, int64_t N, int group, int sym,
 
 /*
  * w4a16_workspace_bytes -- scratch bytes w4a16_gemm needs for this shape
- * (0 when it needs none).  The workspace holds split-K partial sums and
- * per-tile arrival counters; it must be zero-filled once before its first
- * use, and w4a16_gemm leaves it zero-filled again when its work completes,
- * so one workspace can serve any number of calls issued on ONE stream
- * (calls that may overlap need separate workspaces).
+ * (0 when it needs none).  The workspace holds per-tile arrival counters
+ * (a fixed area at its start) and split-K partial sums.  It must be
+ * zero-filled once before its first use; every w4a16_gemm call leaves the
+ * counter area zero again when its work completes and fully rewrites the
+ * partials it reads, so one workspace serves any number of calls of any
+ * shapes issued one after another on ONE stream.  Calls that may overlap on
+ * the GPU (other streams) need separate workspaces.
  */
 size_t w4a16_workspace_bytes(int64_t M, int64_t K, int64_t N, int group);
 

@@ -45,6 +45,13 @@ constexpr int kGroup = 128;
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kBatch = 4;  // groups whose weight loads are in flight together
+// Workspace layout when K is split across CTAs: a fixed area of arrival
+// counters first (one per row block), then the fp32 partials.  The counters
+// sit at the same place for every shape, so a workspace shared by calls of
+// different shapes stays valid: every call leaves its counters at zero and
+// fully overwrites the partials it reads.
+constexpr int kMaxCounters = 1024;
+constexpr size_t kCounterBytes = kMaxCounters * sizeof(unsigned);
 
 struct DecodeCfg {
     int MT, RT, WN;  // n8 tiles of X rows, 16-row weight tiles per warp, warps along N
@@ -344,9 +351,10 @@ int make_plan(int64_t M, int64_t K, int64_t N, Plan *p) {
     if (want > maxs) want = maxs;
     if (want > 16) want = 16;
     p->splits = want < 1 ? 1 : want;
+    if (p->row_blocks > kMaxCounters) p->splits = 1;
     if (p->splits > 1) {
         p->partial_bytes = ((size_t)p->splits * M * N * sizeof(float) + 255) & ~(size_t)255;
-        p->count_bytes = ((size_t)p->row_blocks * sizeof(unsigned) + 15) & ~(size_t)15;
+        p->count_bytes = kCounterBytes;
     } else {
         p->partial_bytes = p->count_bytes = 0;
     }
@@ -359,8 +367,8 @@ int launch_t(const Plan &p, const void *X, int64_t M, const uint8_t *packed, con
     float *partial = nullptr;
     unsigned *count = nullptr;
     if (p.splits > 1) {
-        partial = static_cast<float *>(ws);
-        count = reinterpret_cast<unsigned *>(static_cast<char *>(ws) + p.partial_bytes);
+        count = static_cast<unsigned *>(ws);
+        partial = reinterpret_cast<float *>(static_cast<char *>(ws) + p.count_bytes);
     }
     dim3 grid(p.row_blocks, p.splits);
     decode_kernel<XT, MT, RT, WN><<<grid, kThreads, 0, stream>>>(

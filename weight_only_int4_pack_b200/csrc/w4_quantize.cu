@@ -197,7 +197,9 @@ quantize_kernel(const uint16_t *__restrict__ W, int64_t K, int64_t N,
                     }
                     s = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
                     zp = 0.0f;
-                    if (s != 0.0f) zp = fminf(fmaxf(rintf(__fdiv_rn(-mn, s)), 0.0f), 15.0f);
+                    // "+ 0" stores an integer zero point of 0 as +0.0, never -0.0
+                    if (s != 0.0f)
+                        zp = __fadd_rn(fminf(fmaxf(rintf(__fdiv_rn(-mn, s)), 0.0f), 15.0f), 0.0f);
                 }
                 uint32_t bits[8];
                 if (s == 0.0f) {
