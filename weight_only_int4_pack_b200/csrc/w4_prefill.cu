@@ -256,8 +256,43 @@ struct Smem {
     int abort_flag;
 };
 
+// Dequantizes the two stages of group g of the current tile (stage counter
+// base `it`) for this thread's A-tile row dr, k half dkh: waits for the codes,
+// writes 4 swizzled 16-byte chunks per stage, fences them for the tensor
+// core and arrives on the stage's A-ready barrier.
 template <int XT>
-__global__ void __launch_bounds__(kThreads, 1)
+__device__ __forceinline__ bool dequant_group(int g, uint32_t it, int n_d, int G,
+                                              const float *__restrict__ zeros, const uint8_t *cs,
+                                              uint8_t *as, int dr, int dkh, Smem *sm,
+                                              volatile int *abort_flag, unsigned *status) {
+    const float z = zeros ? __ldg(zeros + (int64_t)n_d * G + g) : 8.0f;
+    uint32_t zb, zq;
+    zero_bias<XT>(z, zb, zq);
+#pragma unroll
+    for (int h = 0; h < kGroup / kBK; ++h) {
+        const uint32_t j = it + (uint32_t)(g * (kGroup / kBK) + h);
+        const int s = j % kStages;
+        const uint32_t ph = (j / kStages) & 1;
+        // warp-uniform outcome: the warp either goes on together or leaves together
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm->full[s]), ph, abort_flag, status)))
+            return false;
+        const uint4 w =
+            *reinterpret_cast<const uint4 *>(cs + s * kCodeTileBytes + dr * (kBK / 2) + dkh * 16);
+        uint8_t *arow = as + s * kATileBytes + dr * 128;
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const int chunk = (dkh * 4 + jj) ^ (dr & 7);
+            *reinterpret_cast<uint4 *>(arow + chunk * 16) = dequant_word<XT>(ws[jj], zb, zq);
+        }
+        fence_proxy_async();
+        mbar_arrive(smem_u32(&sm->aready[s]));
+    }
+    return true;
+}
+
+template <int XT>
+__global__ void __maxnreg__(200)
 prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                const float *__restrict__ scales, const float *__restrict__ zeros, int M, int N,
                int K, void *__restrict__ Y, unsigned *__restrict__ status) {
@@ -332,6 +367,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                 }
             }
         }
+        __syncwarp();  // the whole warp reconverges before the CTA barrier
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
@@ -379,6 +415,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                 }
             }
         }
+        __syncwarp();  // the whole warp reconverges before the CTA barrier
     } else {
         // ---------------- math warps: dequant + epilogue ----------------
         const int mw = warp - 2;             // 0..7
@@ -402,48 +439,34 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
 #pragma unroll
             for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
 
-            // dequantize the stages of group 0 ahead of the first epilogue pass
-            int next_dq_group = 0;
-            auto dequant_group = [&](int g) -> bool {
-                const float z = zeros ? __ldg(zeros + (int64_t)n_d * G + g) : 8.0f;
-                uint32_t zb, zq;
-                zero_bias<XT>(z, zb, zq);
-                for (int h = 0; h < kGroup / kBK; ++h) {
-                    const uint32_t j = it + (uint32_t)(g * (kGroup / kBK) + h);
-                    const int s = j % kStages;
-                    const uint32_t ph = (j / kStages) & 1;
-                    if (!mbar_wait(smem_u32(&sm->full[s]), ph, abort_flag, status)) return false;
-                    const uint4 w = *reinterpret_cast<const uint4 *>(cs + s * kCodeTileBytes +
-                                                                      dr * (kBK / 2) + dkh * 16);
-                    uint8_t *arow = as + s * kATileBytes + dr * 128;
-                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        const int chunk = (dkh * 4 + jj) ^ (dr & 7);
-                        *reinterpret_cast<uint4 *>(arow + chunk * 16) = dequant_word<XT>(ws[jj], zb, zq);
-                    }
-                    fence_proxy_async();
-                    mbar_arrive(smem_u32(&sm->aready[s]));
-                }
-                return true;
-            };
-
             // Stay at most one group ahead with the dequantization: the ring holds
             // kStages = 2 groups of stages, and a stage can only be refilled once
             // the MMAs of the group before it have run.
-            if (!dequant_group(0)) { ok = false; break; }
+            int next_dq_group = 0;
+            if (!dequant_group<XT>(0, it, n_d, G, zeros, cs, as, dr, dkh, sm, abort_flag, status)) {
+                ok = false;
+                break;
+            }
             next_dq_group = 1;
             float s_next = __ldg(scales + (int64_t)n_ec * G + 0);
             for (int g = 0; g < G; ++g, ++gc) {
                 if (next_dq_group < G) {
-                    if (!dequant_group(next_dq_group)) { ok = false; break; }
+                    if (!dequant_group<XT>(next_dq_group, it, n_d, G, zeros, cs, as, dr, dkh, sm,
+                                           abort_flag, status)) {
+                        ok = false;
+                        break;
+                    }
                     ++next_dq_group;
                 }
                 const float sg = s_next;
                 if (g + 1 < G) s_next = __ldg(scales + (int64_t)n_ec * G + g + 1);
                 const int b = gc & 1;
                 const uint32_t pph = (gc >> 1) & 1;
-                if (!mbar_wait(smem_u32(&sm->pfull[b]), pph, abort_flag, status)) { ok = false; break; }
+                if (!__all_sync(0xffffffffu,
+                                mbar_wait(smem_u32(&sm->pfull[b]), pph, abort_flag, status))) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
                 const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16) +
                                        static_cast<uint32_t>(b * kBN + colhalf * 128);
@@ -463,7 +486,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             // store this thread's row n_e for its 128 columns m
             if (n_e < N) {
                 const int m0 = mt * kBN + colhalf * 128;
-#pragma unroll 8
+#pragma unroll
                 for (int i = 0; i < 128; ++i) {
                     const int m = m0 + i;
                     if (m < M) store_y<XT>(Y, (int64_t)m * N + n_e, acc[i]);
@@ -530,12 +553,14 @@ int launch_t(const void *X, int64_t M, const uint8_t *packed, const float *scale
                      (uint64_t)K / 2, kBK / 2, kBM, CU_TENSOR_MAP_SWIZZLE_NONE))
         return W4_ERR_CUDA;
     auto kern = prefill_kernel<XT>;
-    static bool attr_done[2] = {false, false};
-    if (!attr_done[XT]) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return W4_ERR_CUDA;
+    static bool attr_done[64][2] = {};
+    if (!attr_done[dev][XT]) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
             cudaSuccess)
             return W4_ERR_CUDA;
-        attr_done[XT] = true;
+        attr_done[dev][XT] = true;
     }
     const int64_t tiles = ((N + kBM - 1) / kBM) * ((M + kBN - 1) / kBN);
     const int grid = (int)(tiles < di.sm_count ? tiles : di.sm_count);
