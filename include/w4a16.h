@@ -126,6 +126,14 @@ int w4a16_gemm(const void *X, int xt, int64_t M, const uint8_t *packed, const fl
  */
 int w4_device_status(int reset);
 
+/*
+ * w4_last_error -- text describing the most recent failure on the calling
+ * thread: which check or which CUDA call failed, and why ("" if none yet).
+ * Thread-local storage owned by the library, valid until the thread's next
+ * failing call; never NULL.
+ */
+const char *w4_last_error(void);
+
 /* Human-readable name of a status code (static storage; never NULL). */
 const char *w4_status_string(int status);
 

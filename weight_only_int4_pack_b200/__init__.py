@@ -25,6 +25,7 @@ import torch
 __all__ = [
     "W4Error", "load", "lib_path", "w4_quantize", "w4_quantize_into", "w4a16_workspace_bytes",
     "w4a16_gemm", "w4a16_gemm_into", "w4_status_string", "w4_device_status", "w4_abi_version",
+    "w4_last_error",
     "Workspace", "W4_OK", "W4_ERR_INVALID_ARG", "W4_ERR_UNSUPPORTED", "W4_ERR_CUDA",
     "W4_ERR_TIMEOUT", "W4_F16", "W4_BF16",
 ]
@@ -40,7 +41,12 @@ _lib = None
 class W4Error(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
-        super().__init__(f"{fn} failed: {w4_status_string(status)} ({status})")
+        detail = ""
+        try:
+            detail = load().w4_last_error().decode()
+        except Exception:
+            pass
+        super().__init__(f"{fn} failed: {w4_status_string(status)} ({status}) {detail}".rstrip())
 
 
 def load() -> ctypes.CDLL:
@@ -65,6 +71,8 @@ def load() -> ctypes.CDLL:
     lib.w4_status_string.restype = ctypes.c_char_p
     lib.w4_abi_version.argtypes = []
     lib.w4_abi_version.restype = I
+    lib.w4_last_error.argtypes = []
+    lib.w4_last_error.restype = ctypes.c_char_p
     _lib = lib
     return lib
 
@@ -101,6 +109,11 @@ def w4_status_string(status: int) -> str:
         return load().w4_status_string(int(status)).decode()
     except RuntimeError:
         return str(status)
+
+
+def w4_last_error() -> str:
+    """Description of the last failure on this thread (which check or CUDA call)."""
+    return load().w4_last_error().decode()
 
 
 def w4_abi_version() -> int:

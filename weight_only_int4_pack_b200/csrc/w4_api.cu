@@ -1,6 +1,9 @@
 // w4_api.cu -- the extern "C" entry points of libw4a16.so (declared in
 // include/w4a16.h): host-side argument validation, dispatch to the kernels,
-// the per-device attribute cache and the device status word.
+// the per-device attribute cache, the device status word and the
+// thread-local description of the last failure.
+
+#include <stdio.h>
 
 #include <mutex>
 
@@ -17,26 +20,43 @@ w4::DeviceInfo g_info[kMaxDevices];
 bool g_info_ok[kMaxDevices] = {};
 unsigned *g_status_ptr[kMaxDevices] = {};
 
+thread_local char g_last_error[320] = "";
+
 bool valid_dtype(int t) { return t == W4_F16 || t == W4_BF16; }
+
+int reject(int status, const char *fn, const char *why) { return w4::set_error(status, fn, why); }
 
 }  // namespace
 
 namespace w4 {
 
+int set_error(int status, const char *what, const char *detail) {
+    if (status != W4_OK)
+        snprintf(g_last_error, sizeof g_last_error, "%s: %s%s%s", w4_status_string(status), what,
+                 detail ? ": " : "", detail ? detail : "");
+    return status;
+}
+
+int cuda_fail(const char *what, cudaError_t e) {
+    return set_error(W4_ERR_CUDA, what, cudaGetErrorString(e));
+}
+
 int device_info(DeviceInfo *out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return W4_ERR_CUDA;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    if (dev < 0 || dev >= kMaxDevices) return set_error(W4_ERR_CUDA, "device ordinal", "out of range");
     std::lock_guard<std::mutex> lk(g_mu);
     if (!g_info_ok[dev]) {
         DeviceInfo d;
         int l2 = 0;
-        if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
-                cudaSuccess ||
-            cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess)
-            return W4_ERR_CUDA;
+        if ((e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                                        dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev)) != cudaSuccess)
+            return cuda_fail("cudaDeviceGetAttribute", e);
         d.l2_bytes = static_cast<size_t>(l2);
         g_info[dev] = d;
         g_info_ok[dev] = true;
@@ -51,7 +71,11 @@ unsigned *device_status_ptr() {
     std::lock_guard<std::mutex> lk(g_mu);
     if (!g_status_ptr[dev]) {
         void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_w4_status) != cudaSuccess) return nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_w4_status);
+        if (e != cudaSuccess) {
+            cuda_fail("cudaGetSymbolAddress(status word)", e);
+            return nullptr;
+        }
         g_status_ptr[dev] = static_cast<unsigned *>(p);
     }
     return g_status_ptr[dev];
@@ -59,9 +83,65 @@ unsigned *device_status_ptr() {
 
 }  // namespace w4
 
+namespace {
+
+int quantize_impl(const void *W, int wt, int64_t K, int64_t N, int group, int sym,
+                  const float *col_scale, uint8_t *packed, float *scales, float *zeros,
+                  void *stream) {
+    const char *fn = "w4_quantize";
+    if (!valid_dtype(wt)) return reject(W4_ERR_INVALID_ARG, fn, "wt is not W4_F16 or W4_BF16");
+    if (K <= 0 || N < 0) return reject(W4_ERR_INVALID_ARG, fn, "K must be > 0 and N >= 0");
+    if (group <= 0 || K % group != 0)
+        return reject(W4_ERR_INVALID_ARG, fn, "K must be a positive multiple of group");
+    if (K % 8 != 0) return reject(W4_ERR_INVALID_ARG, fn, "K must be a multiple of 8");
+    if (N > (int64_t(1) << 40) / K) return reject(W4_ERR_INVALID_ARG, fn, "N * K too large");
+    if (N == 0) return W4_OK;
+    if (!W || !packed || !scales || !zeros) return reject(W4_ERR_INVALID_ARG, fn, "null pointer");
+    if (group != 32 && group != 64 && group != 128 && group != 256)
+        return reject(W4_ERR_UNSUPPORTED, fn, "group must be 32, 64, 128 or 256");
+    if (!w4::aligned16(W) || !w4::aligned16(packed) || !w4::aligned16(scales) ||
+        !w4::aligned16(zeros) || (col_scale && !w4::aligned16(col_scale)))
+        return reject(W4_ERR_UNSUPPORTED, fn, "pointers must be 16-byte aligned");
+    return w4::launch_quantize(W, wt, K, N, group, sym, col_scale, packed, scales, zeros,
+                               static_cast<cudaStream_t>(stream));
+}
+
+int gemm_impl(const void *X, int xt, int64_t M, const uint8_t *packed, const float *scales,
+              const float *zeros, int64_t K, int64_t N, int group, void *Y, void *workspace,
+              size_t workspace_bytes, void *stream) {
+    const char *fn = "w4a16_gemm";
+    if (!valid_dtype(xt)) return reject(W4_ERR_INVALID_ARG, fn, "xt is not W4_F16 or W4_BF16");
+    if (M < 0 || K <= 0 || N < 0) return reject(W4_ERR_INVALID_ARG, fn, "need M >= 0, K > 0, N >= 0");
+    if (group <= 0 || K % group != 0)
+        return reject(W4_ERR_INVALID_ARG, fn, "K must be a positive multiple of group");
+    if (K % 8 != 0) return reject(W4_ERR_INVALID_ARG, fn, "K must be a multiple of 8");
+    if (M > (int64_t(1) << 31) || N > (int64_t(1) << 31) || K > (int64_t(1) << 31))
+        return reject(W4_ERR_INVALID_ARG, fn, "M, N and K must be below 2^31");
+    if (M == 0 || N == 0) return W4_OK;
+    if (!X || !packed || !scales || !Y) return reject(W4_ERR_INVALID_ARG, fn, "null pointer");
+    if (group != 128) return reject(W4_ERR_UNSUPPORTED, fn, "group must be 128");
+    if (!w4::aligned16(X) || !w4::aligned16(packed) || !w4::aligned16(scales) ||
+        (zeros && !w4::aligned16(zeros)) || !w4::aligned16(Y))
+        return reject(W4_ERR_UNSUPPORTED, fn, "pointers must be 16-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M <= 32) {
+        const size_t need = w4::decode_workspace_bytes(M, K, N, group);
+        if (need > 0 && (!workspace || workspace_bytes < need || !w4::aligned16(workspace)))
+            return reject(W4_ERR_INVALID_ARG, fn,
+                          "workspace missing, misaligned or smaller than w4a16_workspace_bytes");
+        return w4::launch_decode(X, xt, M, packed, scales, zeros, K, N, Y, workspace,
+                                 workspace_bytes, s);
+    }
+    return w4::launch_prefill(X, xt, M, packed, scales, zeros, K, N, Y, s);
+}
+
+}  // namespace
+
 extern "C" {
 
 int w4_abi_version(void) { return W4A16_ABI_VERSION; }
+
+const char *w4_last_error(void) { return g_last_error; }
 
 const char *w4_status_string(int status) {
     switch (status) {
@@ -77,17 +157,7 @@ const char *w4_status_string(int status) {
 int w4_quantize(const void *W, int wt, int64_t K, int64_t N, int group, int sym,
                 const float *col_scale, uint8_t *packed, float *scales, float *zeros,
                 void *stream) {
-    if (!valid_dtype(wt) || K <= 0 || N < 0 || group <= 0) return W4_ERR_INVALID_ARG;
-    if (K % group != 0 || K % 8 != 0) return W4_ERR_INVALID_ARG;
-    if (N > (int64_t(1) << 40) / K) return W4_ERR_INVALID_ARG;
-    if (N == 0) return W4_OK;
-    if (!W || !packed || !scales || !zeros) return W4_ERR_INVALID_ARG;
-    if (group != 32 && group != 64 && group != 128 && group != 256) return W4_ERR_UNSUPPORTED;
-    if (!w4::aligned16(W) || !w4::aligned16(packed) || !w4::aligned16(scales) ||
-        !w4::aligned16(zeros) || (col_scale && !w4::aligned16(col_scale)))
-        return W4_ERR_UNSUPPORTED;
-    return w4::launch_quantize(W, wt, K, N, group, sym, col_scale, packed, scales, zeros,
-                               static_cast<cudaStream_t>(stream));
+    return quantize_impl(W, wt, K, N, group, sym, col_scale, packed, scales, zeros, stream);
 }
 
 size_t w4a16_workspace_bytes(int64_t M, int64_t K, int64_t N, int group) {
@@ -99,33 +169,20 @@ size_t w4a16_workspace_bytes(int64_t M, int64_t K, int64_t N, int group) {
 int w4a16_gemm(const void *X, int xt, int64_t M, const uint8_t *packed, const float *scales,
                const float *zeros, int64_t K, int64_t N, int group, void *Y, void *workspace,
                size_t workspace_bytes, void *stream) {
-    if (!valid_dtype(xt) || M < 0 || K <= 0 || N < 0 || group <= 0) return W4_ERR_INVALID_ARG;
-    if (K % group != 0 || K % 8 != 0) return W4_ERR_INVALID_ARG;
-    if (M > (int64_t(1) << 31) || N > (int64_t(1) << 31) || K > (int64_t(1) << 31))
-        return W4_ERR_INVALID_ARG;
-    if (M == 0 || N == 0) return W4_OK;
-    if (!X || !packed || !scales || !Y) return W4_ERR_INVALID_ARG;
-    if (group != 128) return W4_ERR_UNSUPPORTED;
-    if (!w4::aligned16(X) || !w4::aligned16(packed) || !w4::aligned16(scales) ||
-        (zeros && !w4::aligned16(zeros)) || !w4::aligned16(Y))
-        return W4_ERR_UNSUPPORTED;
-    const size_t need = w4a16_workspace_bytes(M, K, N, group);
-    if (need > 0 && (!workspace || workspace_bytes < need || !w4::aligned16(workspace)))
-        return W4_ERR_INVALID_ARG;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (M <= 32)
-        return w4::launch_decode(X, xt, M, packed, scales, zeros, K, N, Y, workspace,
-                                 workspace_bytes, s);
-    return w4::launch_prefill(X, xt, M, packed, scales, zeros, K, N, Y, s);
+    return gemm_impl(X, xt, M, packed, scales, zeros, K, N, group, Y, workspace, workspace_bytes,
+                     stream);
 }
 
 int w4_device_status(int reset) {
-    if (cudaDeviceSynchronize() != cudaSuccess) return W4_ERR_CUDA;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return w4::cuda_fail("cudaDeviceSynchronize", e);
     unsigned v = 0;
-    if (cudaMemcpyFromSymbol(&v, g_w4_status, sizeof v) != cudaSuccess) return W4_ERR_CUDA;
+    if ((e = cudaMemcpyFromSymbol(&v, g_w4_status, sizeof v)) != cudaSuccess)
+        return w4::cuda_fail("read status word", e);
     if (reset) {
         const unsigned zero = 0;
-        if (cudaMemcpyToSymbol(g_w4_status, &zero, sizeof zero) != cudaSuccess) return W4_ERR_CUDA;
+        if ((e = cudaMemcpyToSymbol(g_w4_status, &zero, sizeof zero)) != cudaSuccess)
+            return w4::cuda_fail("clear status word", e);
     }
     return v ? W4_ERR_TIMEOUT : W4_OK;
 }

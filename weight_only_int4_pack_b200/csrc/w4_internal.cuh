@@ -23,7 +23,12 @@ int device_info(DeviceInfo *out);  // W4_OK or W4_ERR_CUDA
 // (kernels set W4_ERR_TIMEOUT into it when a bounded wait runs out).
 unsigned *device_status_ptr();
 
-inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? W4_OK : W4_ERR_CUDA; }
+// Records a description of the failing call for w4_last_error() and
+// returns the status.  `what` names the call; `detail` may be null.
+int set_error(int status, const char *what, const char *detail);
+int cuda_fail(const char *what, cudaError_t e);  // W4_ERR_CUDA with the runtime's text
+
+inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? W4_OK : cuda_fail("kernel launch", e); }
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

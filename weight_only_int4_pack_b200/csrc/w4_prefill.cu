@@ -42,6 +42,8 @@
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
+#include <stdio.h>
+
 #include <mutex>
 
 #include "w4_internal.cuh"
@@ -190,6 +192,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -292,7 +304,7 @@ __device__ __forceinline__ bool dequant_group(int g, uint32_t it, int n_d, int G
 }
 
 template <int XT>
-__global__ void __maxnreg__(200)
+__global__ void __maxnreg__(184)
 prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                const float *__restrict__ scales, const float *__restrict__ zeros, int M, int N,
                int K, void *__restrict__ Y, unsigned *__restrict__ status) {
@@ -471,12 +483,13 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                 const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16) +
                                        static_cast<uint32_t>(b * kBN + colhalf * 128);
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(taddr + 32 * c, r);
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t r[16];
+                    tmem_ld16(taddr + 16 * c, r);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) acc[32 * c + i] = fmaf(sg, __uint_as_float(r[i]), acc[32 * c + i]);
+                    for (int i = 0; i < 16; ++i)
+                        acc[16 * c + i] = fmaf(sg, __uint_as_float(r[i]), acc[16 * c + i]);
                 }
                 tc_fence_before();
                 mbar_arrive(smem_u32(&sm->pempty[b]));
@@ -511,20 +524,20 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static std::once_flag once;
     std::call_once(once, [] {
         void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
             fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
     });
     return fn;
 }
 
-bool make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *ptr, uint64_t inner,
-                 uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
-                 CUtensorMapSwizzle swz) {
+int make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *ptr, uint64_t inner,
+                uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                CUtensorMapSwizzle swz, const char *what) {
     auto fn = encode_fn();
-    if (!fn) return false;
+    if (!fn) return set_error(W4_ERR_CUDA, what, "cuTensorMapEncodeTiled entry point not found");
     cuuint64_t dims[2] = {inner, outer};
     cuuint64_t strides[1] = {row_bytes};
     cuuint32_t box[2] = {box_inner, box_outer};
@@ -532,7 +545,12 @@ bool make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *ptr, uint
     CUresult r = fn(map, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    if (r != CUDA_SUCCESS) {
+        char buf[64];
+        snprintf(buf, sizeof buf, "cuTensorMapEncodeTiled returned CUresult %d", (int)r);
+        return set_error(W4_ERR_CUDA, what, buf);
+    }
+    return W4_OK;
 }
 
 template <int XT>
@@ -541,26 +559,44 @@ int launch_t(const void *X, int64_t M, const uint8_t *packed, const float *scale
     DeviceInfo di;
     int st = device_info(&di);
     if (st != W4_OK) return st;
-    if (di.cc_major != 10) return W4_ERR_UNSUPPORTED;
-    if (di.max_smem_optin < kSmemBytes) return W4_ERR_UNSUPPORTED;
+    if (di.cc_major != 10)
+        return set_error(W4_ERR_UNSUPPORTED, "w4a16_gemm (M > 32)", "needs an sm_100 GPU");
+    if (di.max_smem_optin < kSmemBytes)
+        return set_error(W4_ERR_UNSUPPORTED, "w4a16_gemm (M > 32)", "not enough shared memory");
     unsigned *status = device_status_ptr();
     if (!status) return W4_ERR_CUDA;
     CUtensorMap mx, mw;
-    if (!make_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_UINT16, X, (uint64_t)K, (uint64_t)M,
-                     (uint64_t)K * 2, kBK, kBN, CU_TENSOR_MAP_SWIZZLE_128B))
-        return W4_ERR_CUDA;
-    if (!make_map_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)K / 2, (uint64_t)N,
-                     (uint64_t)K / 2, kBK / 2, kBM, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return W4_ERR_CUDA;
+    if ((st = make_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_UINT16, X, (uint64_t)K, (uint64_t)M,
+                          (uint64_t)K * 2, kBK, kBN, CU_TENSOR_MAP_SWIZZLE_128B, "tensor map of X")) !=
+        W4_OK)
+        return st;
+    if ((st = make_map_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)K / 2, (uint64_t)N,
+                          (uint64_t)K / 2, kBK / 2, kBM, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          "tensor map of packed")) != W4_OK)
+        return st;
     auto kern = prefill_kernel<XT>;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return W4_ERR_CUDA;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return set_error(W4_ERR_CUDA, "cudaGetDevice", nullptr);
     static bool attr_done[64][2] = {};
     if (!attr_done[dev][XT]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
-            cudaSuccess)
-            return W4_ERR_CUDA;
+        cudaError_t e =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(prefill smem)", e);
         attr_done[dev][XT] = true;
+    }
+    static int threads_ok[64][2] = {};
+    if (!threads_ok[dev][XT]) {
+        cudaFuncAttributes fa;
+        cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+        if (e != cudaSuccess) return cuda_fail("cudaFuncGetAttributes(prefill)", e);
+        if (fa.maxThreadsPerBlock < kThreads) {
+            char buf[96];
+            snprintf(buf, sizeof buf, "%d registers per thread allow only %d threads", fa.numRegs,
+                     fa.maxThreadsPerBlock);
+            return set_error(W4_ERR_CUDA, "prefill kernel resources", buf);
+        }
+        threads_ok[dev][XT] = 1;
     }
     const int64_t tiles = ((N + kBM - 1) / kBM) * ((M + kBN - 1) / kBN);
     const int grid = (int)(tiles < di.sm_count ? tiles : di.sm_count);

@@ -235,8 +235,8 @@ int launch_t(const void *W, int64_t K, int64_t N, const float *col_scale, uint8_
     static int blocks_per_sm = 0;  // same for every device of one architecture
     if (blocks_per_sm == 0) {
         int b = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, kThreads, 0) != cudaSuccess)
-            return W4_ERR_CUDA;
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, kThreads, 0);
+        if (e != cudaSuccess) return cuda_fail("cudaOccupancyMaxActiveBlocksPerMultiprocessor", e);
         blocks_per_sm = b > 0 ? b : 1;
     }
     const int64_t tiles_k = (K + kStripK - 1) / kStripK;
