@@ -31,6 +31,10 @@
 //               TMEM lane quarter, 128 columns each).  After the last group
 //               of a tile they round acc to the output dtype and store Y.
 //
+// Registers: each SM sub-partition has 16K registers and this 10-warp CTA puts
+// three warps on two of them, so a thread may hold at most 168 registers
+// (the math warps keep 128 fp32 accumulators).
+//
 // Every wait on an mbarrier is bounded (kWaitNs); a wait that runs out sets
 // the library's device status word to W4_ERR_TIMEOUT and a shared abort
 // flag, every role then leaves its loop, the producer and the MMA issuer
@@ -180,18 +184,6 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
                  : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
-        "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-}
-
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
@@ -304,7 +296,7 @@ __device__ __forceinline__ bool dequant_group(int g, uint32_t it, int n_d, int G
 }
 
 template <int XT>
-__global__ void __maxnreg__(184)
+__global__ void __maxnreg__(168)
 prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                const float *__restrict__ scales, const float *__restrict__ zeros, int M, int N,
                int K, void *__restrict__ Y, unsigned *__restrict__ status) {
