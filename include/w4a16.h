@@ -120,6 +120,31 @@ int w4a16_gemm(const void *X, int xt, int64_t M, const uint8_t *packed, const fl
                size_t workspace_bytes, void *stream);
 
 /*
+ * w4a16_gemm_noalloc -- the decode path of w4a16_gemm (M <= 32) for callers
+ * that cannot allocate device memory, such as a plugin inside a host
+ * application that owns every device allocation, or a latency-critical path
+ * where cudaMalloc and the synchronization it may imply are not allowed.  The
+ * source pages have no counterpart to this entry point: it is a property of
+ * this library's interface, not of the method.
+ *
+ *   Arguments and result as w4a16_gemm, without the workspace: the scratch
+ *   space lives in a 4 MiB device array inside the library, which every GPU
+ *   that loads the library holds until the process exits.  The call allocates
+ *   nothing (no cudaMalloc, cudaFree or allocating library routine); it clears
+ *   the counter area of the array with cudaMemsetAsync on `stream` first.
+ *   M > 32 returns W4_ERR_UNSUPPORTED (that path of w4a16_gemm needs no
+ *   workspace); a shape whose workspace would exceed 4 MiB returns
+ *   W4_ERR_UNSUPPORTED, with the reason in w4_last_error().
+ *   All calls on a device share the one array: calls that may overlap on the
+ *   GPU (other streams, other host threads) race and give wrong results.
+ *   The first call on each device looks up the array's device address with
+ *   that device current; make that first call before any stream capture.
+ */
+int w4a16_gemm_noalloc(const void *X, int xt, int64_t M, const uint8_t *packed,
+                       const float *scales, const float *zeros, int64_t K, int64_t N, int group,
+                       void *Y, void *stream);
+
+/*
  * w4_device_status -- reads (and, if reset != 0, clears) the current device's
  * status word that kernels set when a bounded wait runs out.  Synchronizes the
  * device first.  Returns W4_OK, W4_ERR_TIMEOUT, or W4_ERR_CUDA if the read fails.

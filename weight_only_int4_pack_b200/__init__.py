@@ -25,7 +25,7 @@ import torch
 __all__ = [
     "W4Error", "load", "lib_path", "w4_quantize", "w4_quantize_into", "w4a16_workspace_bytes",
     "w4a16_gemm", "w4a16_gemm_into", "w4_status_string", "w4_device_status", "w4_abi_version",
-    "w4_last_error",
+    "w4_last_error", "w4a16_gemm_noalloc",
     "Workspace", "W4_OK", "W4_ERR_INVALID_ARG", "W4_ERR_UNSUPPORTED", "W4_ERR_CUDA",
     "W4_ERR_TIMEOUT", "W4_F16", "W4_BF16",
 ]
@@ -71,6 +71,8 @@ def load() -> ctypes.CDLL:
     lib.w4_status_string.restype = ctypes.c_char_p
     lib.w4_abi_version.argtypes = []
     lib.w4_abi_version.restype = I
+    lib.w4a16_gemm_noalloc.argtypes = [P, I, I64, P, P, P, I64, I64, I, P, P]
+    lib.w4a16_gemm_noalloc.restype = I
     lib.w4_last_error.argtypes = []
     lib.w4_last_error.restype = ctypes.c_char_p
     _lib = lib
@@ -198,3 +200,18 @@ def w4a16_gemm(X, packed, scales, zeros=None, group: int = 128, out=None, worksp
     N = packed.shape[0]
     Y = out if out is not None else torch.empty((M, N), dtype=X.dtype, device=X.device)
     return w4a16_gemm_into(X, packed, scales, zeros, Y, group, workspace, stream)
+
+
+def w4a16_gemm_noalloc(X, packed, scales, zeros=None, group: int = 128, out=None, stream=None):
+    """The decode layer (M <= 32) with the library's own static scratch space:
+    for callers that cannot allocate device memory.  Calls on one device must
+    not overlap on the GPU (they share that scratch space)."""
+    _check_dev(X, packed, scales, zeros, out)
+    M, K = X.shape
+    N = packed.shape[0]
+    Y = out if out is not None else torch.empty((M, N), dtype=X.dtype, device=X.device)
+    st = load().w4a16_gemm_noalloc(_p(X), _dt(X), M, _p(packed), _p(scales), _p(zeros), K, N,
+                                   int(group), _p(Y), _stream(stream))
+    if st != W4_OK:
+        raise W4Error("w4a16_gemm_noalloc", st)
+    return Y
