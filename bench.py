@@ -536,6 +536,51 @@ def workload_config():
 
 # ---------------------------------------------------------------------------- main
 
+def run_profile_case(args):
+    """Runs `--launches` launches of one kernel on its workload, untimed: the
+    command the ncu summaries under profiles/ were taken with."""
+    import weight_only_int4_pack_b200 as w4
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w4.load()
+    case = args.profile
+    if case.startswith("decode"):
+        if case == "decode_m1":
+            c = synth.DECODE_M1
+            M, K, N, sym = 1, c["K"], c["Ns"][-1], c["sym"]
+        else:
+            c = synth.DECODE_SMALLM
+            M, K, N, sym = int(case.split("_m")[-1]), c["K"], c["N"], c["sym"]
+        p, s, z = make_layer(w4, N, K, sym, c["seed"], 4, std=c["std"])
+        X = synth.activations(M, K, c["seed"], salient_frac=0.01, device=dev)
+        Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        torch.cuda.synchronize()
+        for _ in range(args.launches):
+            w4.w4a16_gemm(X, p, s, z, out=Y)
+    elif case == "prefill":
+        c = synth.PREFILL
+        p, s, z = make_layer(w4, c["N"], c["K"], c["sym"], c["seed"], 4, dtype="bf16", std=c["std"])
+        X = synth.activations(c["M"], c["K"], c["seed"], salient_frac=0.01, dtype="bf16", device=dev)
+        torch.cuda.synchronize()
+        for _ in range(args.launches):
+            w4.w4a16_gemm(X, p, s, z)
+    elif case == "quantize":
+        # the largest projection of the 7B stack (gate_up, 22016 x 4096), AWQ factor folded
+        c = synth.STACK_7B
+        W = synth.weights(22016, 4096, c["std"], c["seed"], outlier_frac=c["w_outlier"], device=dev,
+                          tensor_id=18)
+        cs = synth.awq_col_scale(synth.activations(c["calib_M"], 4096, c["seed"],
+                                                   salient_frac=c["x_salient"], tensor_id=2,
+                                                   device=dev))
+        torch.cuda.synchronize()
+        for _ in range(args.launches):
+            w4.w4_quantize(W, GROUP, sym=False, col_scale=cs)
+    else:
+        raise SystemExit(f"unknown --profile case {case}")
+    torch.cuda.synchronize()
+    print(f"profile case {case}: {args.launches} launches done")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -544,7 +589,14 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--sections", default="all")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--profile", default=None,
+                    help="decode_m1 | decode_m4..decode_m32 | prefill | quantize: run --launches "
+                         "launches of that kernel untimed (for ncu)")
+    ap.add_argument("--launches", type=int, default=3)
     args = ap.parse_args()
+    if args.profile:
+        run_profile_case(args)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     ws_, rank, local = dist_info()
