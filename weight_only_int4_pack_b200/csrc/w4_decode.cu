@@ -1,40 +1,49 @@
 // w4_decode.cu -- the W4A16 linear layer for small M (decode, M <= 32).
 //
-// Y[m][n] = sum_k X[m][k] * (u[n][k] - zero[n][g]) * scale[n][g]: the
-// "dequant -> 16-bit matmul" of W4A16 ("Quantization method families",
-// inference-learning-path.pages.dev, §2), with dequantization as in
-// "LLM quantization methods: principles and implementation"
-// (zhiyuanblog.org/blog/llm-quantization) §2.2.  At small M the layer is
-// bound by streaming the packed weights from HBM.
+// Y[m][n] = sum_g scale[n][g] * sum_{k in g} X[m][k] * (u[n][k] - zero[n][g]):
+// the "dequant -> 16-bit matmul" of W4A16 ("Quantization method families",
+// inference-learning-path.pages.dev, §2), dequantization as in "LLM
+// quantization methods: principles and implementation"
+// (zhiyuanblog.org/blog/llm-quantization) §2.2-§2.3.  At small M the layer is
+// bound by streaming the packed weights from HBM, so the kernel is built to
+// keep HBM busy from the first cycle to the last:
 //
-// Design (B200, sm_100a):
-//   * Swap-AB tensor-core GEMV: a warp owns RT tiles of 16 weight rows and
-//     runs mma.sync m16n8k16 with the dequantized weights as the 16-row A
-//     operand and X as the 8-column B operand (M padded to 8*MT).  The A
-//     fragments are built in registers straight from the packed words, so
-//     the weights never touch shared memory.
-//   * Exact operands: (u - zero) is an integer in [-15, 15], exact in fp16
-//     and bf16.  It is produced with the exponent-bias trick (OR the nibble
-//     into the mantissa of 1024.0 (fp16) or 128.0 (bf16), subtract the biased
-//     zero point); the group's fp32 partial sum is multiplied by the group
-//     scale afterwards.  No weight is ever rounded to 16 bits.
-//   * The packed layout puts k = 8j+{0,1} in nibbles 0 and 4 of word j,
-//     k+{2,3} in nibbles 1 and 5, etc., so one mask pulls a pair of
-//     consecutive k into the two halves of a 32-bit register.  Thread (g, t)
-//     of a warp loads the 32 consecutive k = 32t..32t+31 of a group for rows
-//     g and g+8 (one 16-byte load each) and the matching 16 bytes of X per
-//     word, so no register shuffles are needed: mma (word j, half h) maps the
-//     fragment's k indices {2t,2t+1,2t+8,2t+9} to the physical
-//     k = 32t + 8j + 4h + {0,1,2,3}.
-//   * Split-K: the 8 warps of a CTA split K (WK ways) and reduce through
-//     shared memory in a fixed order.  When there are too few row tiles to
-//     fill the GPU, the grid also splits K across CTAs: each CTA writes an
-//     fp32 partial to the caller's workspace and the last CTA to arrive on a
-//     tile (atomic counter) sums the partials in split order, writes Y and
-//     re-arms the counter.  The result is deterministic.
+//   * Persistent, one CTA per SM.  The packed matrix is cut into units of
+//     128 weight rows x 256 k (16 KB of codes).  The units, in row-block-major
+//     order, are split into equal contiguous ranges, one per CTA ("stream-K"):
+//     every SM streams the same number of bytes whatever N and K are.
+//   * A producer warp streams the CTA's units into an 8-stage shared-memory
+//     ring with TMA (128-byte swizzle), up to 128 KB in flight per SM.
+//   * Eight consumer warps each own 16 of the unit's rows and run
+//     mma.sync m16n8k16 "swap-AB": the dequantized weights are the 16-row A
+//     operand, built in registers from the swizzled codes, X is the B operand
+//     (M padded to 8*MT).  The A operand holds (u - zero), an integer in
+//     [-15, 15], exact in fp16/bf16 (exponent-bias trick: OR the nibble into
+//     the mantissa of 1024.0 or 128.0, subtract the biased zero point); the
+//     fp32 partial of each group is multiplied by its scale afterwards, so no
+//     weight is rounded to 16 bits.
+//   * A row block whose units all fall in one CTA's range is written to Y
+//     directly.  A row block split between CTAs: each warp writes its fp32
+//     partial (16 rows) to its CTA's slot in the caller's workspace; the last
+//     warp to arrive on that (row block, warp) counter adds the slots in CTA
+//     order, writes Y and re-arms the counter.  No warp ever waits for
+//     another warp, and the result is deterministic.
+//   * Fragment layout: thread (g, t) holds k = 32t..32t+31 of each group, so
+//     mma (word j, half h) maps the fragment's k indices {2t,2t+1,2t+8,2t+9}
+//     to k = 32t + 8j + 4h + {0,1,2,3}; the packed layout puts consecutive k
+//     pairs in the two halves of one masked 32-bit word, so no shuffles are
+//     needed.  mma row g reads unit row 16w + ((g & 1) << 2 | g >> 1) (and
+//     that + 8): the rows of one 8-lane load phase then differ in bit 2 of
+//     the swizzle key, which makes the 16-byte shared-memory loads
+//     conflict-free.
+//
+// Every mbarrier wait is bounded; a wait that runs out sets the library's
+// status word (W4_ERR_TIMEOUT) and an abort flag, and all warps leave.
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <stdio.h>
+
 
 #include "w4_internal.cuh"
 
@@ -42,33 +51,80 @@ namespace w4 {
 namespace {
 
 constexpr int kGroup = 128;
-constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
-constexpr int kBatch = 4;  // groups whose weight loads are in flight together
-// Workspace layout when K is split across CTAs: a fixed area of arrival
-// counters first (one per row block), then the fp32 partials.  The counters
-// sit at the same place for every shape, so a workspace shared by calls of
-// different shapes stays valid: every call leaves its counters at zero and
-// fully overwrites the partials it reads.
-constexpr int kMaxCounters = 1024;
+constexpr int kUnitRows = 128;                  // weight rows per unit
+constexpr int kUnitK = 256;                     // k per unit (two groups, 128 bytes of codes per row)
+constexpr int kUnitBytes = kUnitRows * kUnitK / 2;  // 16 KB
+constexpr int kStages = 8;
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = 32 * kConsumerWarps;    // 256
+constexpr int kThreads = kConsumers + 32;          // + producer warp
+constexpr int kSmemBytes = kStages * kUnitBytes + 1024 + 256;
+// Workspace: arrival counters (one per row block and consumer warp) first,
+// then two partial slots per CTA ([2 * ctas][128 rows][M] fp32).  The counter
+// area is fixed so that one workspace serves calls of any shape; row-block
+// counts beyond it switch to whole-row-block ranges, which need no workspace.
+constexpr int kMaxRowBlocks = 2048;
+constexpr int kMaxCounters = kMaxRowBlocks * kConsumerWarps;
 constexpr size_t kCounterBytes = kMaxCounters * sizeof(unsigned);
+constexpr unsigned long long kWaitNs = 2000000000ull;
 
-struct DecodeCfg {
-    int MT, RT, WN;  // n8 tiles of X rows, 16-row weight tiles per warp, warps along N
-};
-
-__host__ __device__ constexpr int rows_per_cta(int RT, int WN) { return 16 * RT * WN; }
-
-__device__ __forceinline__ uint4 ldg_stream(const uint32_t *p) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint4 ldg_keep(const void *p) {
-    return __ldg(reinterpret_cast<const uint4 *>(p));
+__device__ __forceinline__ unsigned long long globaltimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                          unsigned *status) {
+    if (mbar_try(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    while (true) {
+        if (mbar_try(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer() - t0 > kWaitNs) {
+            *abort_flag = 1;
+            atomicOr(status, 1u);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
 }
 
 template <int XT>
@@ -88,47 +144,44 @@ __device__ __forceinline__ void mma16816(float d[4], const uint32_t a[4], uint32
     }
 }
 
-// Biased zero point of one row for the current group, in the operand type:
-// fp16: zb = {1024+z, 1024+z}, zq = {-(64+z), -(64+z)}; bf16: zb = {128+z, 128+z}.
+// Biased zero point in the operand type: fp16 zb = {1024+z, 1024+z},
+// zq = {-(64+z), -(64+z)}; bf16 zb = {128+z, 128+z}.
 template <int XT>
-struct ZeroBias {
-    uint32_t zb, zq;
-    __device__ __forceinline__ void set(float z) {
-        if (XT == W4_F16) {
-            __half2 a = __float2half2_rn(1024.0f + z);
-            __half2 b = __float2half2_rn(-(64.0f + z));
-            zb = *reinterpret_cast<uint32_t *>(&a);
-            zq = *reinterpret_cast<uint32_t *>(&b);
-        } else {
-            __nv_bfloat162 a = __float2bfloat162_rn(128.0f + z);
-            zb = *reinterpret_cast<uint32_t *>(&a);
-            zq = 0;
-        }
-    }
-};
-
-// One packed word (k = 8j..8j+7 of a row) -> four registers holding the
-// exact pairs (u-z) of k = {0,1}, {2,3}, {4,5}, {6,7}.
-template <int XT>
-__device__ __forceinline__ void dequant_word(uint32_t w, const ZeroBias<XT> &zb, uint32_t p[4]) {
+__device__ __forceinline__ void zero_bias(float z, uint32_t &zb, uint32_t &zq) {
     if (XT == W4_F16) {
-        const uint32_t magic = 0x64006400u;  // {1024.0, 1024.0}
-        const uint32_t sixteenth = 0x2C002C00u;  // {1/16, 1/16}
-        uint32_t lo0 = (w & 0x000F000Fu) | magic;
-        uint32_t hi0 = (w & 0x00F000F0u) | magic;
-        uint32_t w8 = w >> 8;
-        uint32_t lo1 = (w8 & 0x000F000Fu) | magic;
-        uint32_t hi1 = (w8 & 0x00F000F0u) | magic;
-        asm("sub.f16x2 %0, %1, %2;" : "=r"(p[0]) : "r"(lo0), "r"(zb.zb));
-        asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(p[1]) : "r"(hi0), "r"(sixteenth), "r"(zb.zq));
-        asm("sub.f16x2 %0, %1, %2;" : "=r"(p[2]) : "r"(lo1), "r"(zb.zb));
-        asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(p[3]) : "r"(hi1), "r"(sixteenth), "r"(zb.zq));
+        __half2 a = __float2half2_rn(1024.0f + z);
+        __half2 b = __float2half2_rn(-(64.0f + z));
+        zb = *reinterpret_cast<uint32_t *>(&a);
+        zq = *reinterpret_cast<uint32_t *>(&b);
     } else {
-        const uint32_t magic = 0x43004300u;  // {128.0, 128.0} in bf16
+        __nv_bfloat162 a = __float2bfloat162_rn(128.0f + z);
+        zb = *reinterpret_cast<uint32_t *>(&a);
+        zq = 0;
+    }
+}
+
+// One packed word (k = 8j..8j+7 of a row) -> four registers holding the exact
+// pairs (u - z) of k = {0,1}, {2,3}, {4,5}, {6,7}.
+template <int XT>
+__device__ __forceinline__ void dequant_word(uint32_t w, uint32_t zb, uint32_t zq, uint32_t p[4]) {
+    if (XT == W4_F16) {
+        const uint32_t magic = 0x64006400u;      // {1024, 1024}
+        const uint32_t sixteenth = 0x2C002C00u;  // {1/16, 1/16}
+        const uint32_t lo0 = (w & 0x000F000Fu) | magic;
+        const uint32_t hi0 = (w & 0x00F000F0u) | magic;
+        const uint32_t w8 = w >> 8;
+        const uint32_t lo1 = (w8 & 0x000F000Fu) | magic;
+        const uint32_t hi1 = (w8 & 0x00F000F0u) | magic;
+        asm("sub.f16x2 %0, %1, %2;" : "=r"(p[0]) : "r"(lo0), "r"(zb));
+        asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(p[1]) : "r"(hi0), "r"(sixteenth), "r"(zq));
+        asm("sub.f16x2 %0, %1, %2;" : "=r"(p[2]) : "r"(lo1), "r"(zb));
+        asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(p[3]) : "r"(hi1), "r"(sixteenth), "r"(zq));
+    } else {
+        const uint32_t magic = 0x43004300u;  // {128, 128} in bf16
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            uint32_t v = ((w >> (4 * i)) & 0x000F000Fu) | magic;
-            asm("sub.bf16x2 %0, %1, %2;" : "=r"(p[i]) : "r"(v), "r"(zb.zb));
+            const uint32_t v = ((w >> (4 * i)) & 0x000F000Fu) | magic;
+            asm("sub.bf16x2 %0, %1, %2;" : "=r"(p[i]) : "r"(v), "r"(zb));
         }
     }
 }
@@ -141,272 +194,328 @@ __device__ __forceinline__ void store_out(void *Y, int64_t idx, float v) {
         reinterpret_cast<__nv_bfloat16 *>(Y)[idx] = __float2bfloat16_rn(v);
 }
 
-template <int XT, int MT, int RT, int WN>
-__global__ void __launch_bounds__(kThreads)
-decode_kernel(const uint16_t *__restrict__ X, int M, const uint32_t *__restrict__ packed,
+struct Shared {
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    int abort_flag;
+};
+
+struct Work {
+    int U;       // units in total
+    int KS;      // units per row block
+    int G;       // groups per row
+    int RB;      // row blocks
+    int P;       // CTAs
+    int aligned; // 1: ranges are whole row blocks (no partials)
+};
+
+__host__ __device__ inline int range_start(const Work &w, int c) {
+    if (w.aligned) return (int)((int64_t)c * w.RB / w.P) * w.KS;
+    return (int)((int64_t)c * w.U / w.P);
+}
+
+// CTA whose range holds unit u (stream-K ranges only).
+__device__ __forceinline__ int owner(const Work &w, int u) {
+    return (int)(((int64_t)(u + 1) * w.P - 1) / w.U);
+}
+
+template <int XT, int MT>
+__global__ void __launch_bounds__(kThreads, 1)
+decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__restrict__ X, int M,
               const float *__restrict__ scales, const float *__restrict__ zeros, int K, int N,
-              void *__restrict__ Y, float *__restrict__ ws_partial, unsigned *__restrict__ ws_count,
-              int splits) {
-    constexpr int WK = kWarps / WN;
-    constexpr int ROWS = rows_per_cta(RT, WN);
-    constexpr int MP = 8 * MT;
-    __shared__ float red[WK][ROWS][MP];
-    __shared__ unsigned s_last;
+              void *__restrict__ Y, unsigned *__restrict__ counters, float *__restrict__ partial,
+              const Work wk, unsigned *__restrict__ status) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    Shared *sh = reinterpret_cast<Shared *>(ring + kStages * kUnitBytes);
+    volatile int *abort_flag = &sh->abort_flag;
 
-    const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    const int g = lane >> 2, t = lane & 3;
-    const int wn = warp % WN, wk = warp / WN;
-    const int G = K / kGroup;
-    const int KW = K / 8;  // packed words per row
-    const int rb = blockIdx.x;
-    const int split = blockIdx.y;
-    const int n_cta = rb * ROWS;
-    const int n_warp = n_cta + wn * 16 * RT;
+    const int lane = threadIdx.x & 31;
+    const int c = blockIdx.x;
+    const int u0 = range_start(wk, c);
+    const int u1 = range_start(wk, c + 1);
 
-    // groups of this split, then of this warp
-    const int gs0 = (int)((int64_t)G * split / splits), gs1 = (int)((int64_t)G * (split + 1) / splits);
-    const int gw0 = gs0 + (gs1 - gs0) * wk / WK, gw1 = gs0 + (gs1 - gs0) * (wk + 1) / WK;
-
-    float acc[RT][MT][4];
-#pragma unroll
-    for (int r = 0; r < RT; ++r)
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[r][mt][i] = 0.0f;
-
-    // row pointers of this thread (rows beyond N read row N-1 and are dropped)
-    const uint32_t *wrow[RT][2];
-    int nrow[RT][2];
-#pragma unroll
-    for (int r = 0; r < RT; ++r)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            int n = n_warp + 16 * r + 8 * h + g;
-            nrow[r][h] = n < N ? n : N - 1;
-            wrow[r][h] = packed + (int64_t)nrow[r][h] * KW + 4 * t;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(smem_u32(&sh->full[s]), 1);
+            mbar_init(smem_u32(&sh->empty[s]), kConsumerWarps);
         }
-    // X rows of this thread's B fragments (rows beyond M contribute zero columns)
+        sh->abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    if (warp == kConsumerWarps) {
+        // ---------------- producer ----------------
+        if (lane == 0) {
+            int u = u0;
+            for (; u < u1; ++u) {
+                const int it = u - u0;
+                const int s = it % kStages;
+                const uint32_t ph = (it / kStages) & 1;
+                if (!mbar_wait(smem_u32(&sh->empty[s]), ph ^ 1, abort_flag, status)) break;
+                const uint32_t fb = smem_u32(&sh->full[s]);
+                mbar_arrive_tx(fb, kUnitBytes);
+                const int rb = u / wk.KS, ks = u % wk.KS;
+                tma_load_2d(smem_u32(ring + s * kUnitBytes), &tmap_w, ks * (kUnitK / 2),
+                            rb * kUnitRows, fb);
+            }
+            // wait (bounded) for the copies still in flight before the CTA may exit
+            for (int j = (u - u0 > kStages ? u - u0 - kStages : 0); j < u - u0; ++j) {
+                const unsigned long long t0 = globaltimer();
+                while (!mbar_try(smem_u32(&sh->full[j % kStages]), (j / kStages) & 1) &&
+                       globaltimer() - t0 < kWaitNs) {
+                }
+            }
+        }
+        __syncwarp();
+        return;  // the producer takes no part in the consumers' named barriers
+    }
+
+    // ---------------- consumers ----------------
+    const int g = lane >> 2, t = lane & 3;
+    const int rsel = ((g & 1) << 2) | (g >> 1);  // unit row of mma row g (conflict-free loads)
+    const int lrow0 = 16 * warp + rsel;          // this thread's two rows in the unit
+    const int lrow1 = lrow0 + 8;
+    const int swz = lrow0 & 7;                   // swizzle key of both rows
+    const int G = wk.G;
+
+    // X rows of this thread's B fragments (rows >= M give zero columns)
     const uint16_t *xrow[MT];
     bool xval[MT];
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
-        int m = 8 * mt + g;
+        const int m = 8 * mt + g;
         xval[mt] = m < M;
         xrow[mt] = X + (int64_t)(xval[mt] ? m : 0) * K + 32 * t;
     }
 
-    for (int gb = gw0; gb < gw1; gb += kBatch) {
-        uint4 wv[kBatch][RT][2];
+    float acc[MT][4];
+    int cur_rb = -1, first_ks = 0, last_ks = -1;
+    bool ok = true;
+
+    // Finishes row block rb for this warp's 16 rows.  No step waits on
+    // another warp: a row block split between CTAs has one arrival counter
+    // per (row block, warp), and the last warp to arrive adds the partials.
+    auto flush = [&](int rb) {
+        const int n0 = rb * kUnitRows;
+        if (first_ks == 0 && last_ks == wk.KS - 1) {
 #pragma unroll
-        for (int b = 0; b < kBatch; ++b)
+            for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-            for (int r = 0; r < RT; ++r)
-#pragma unroll
-                for (int h = 0; h < 2; ++h)
-                    if (gb + b < gw1) wv[b][r][h] = ldg_stream(wrow[r][h] + (gb + b) * 16);
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-            const int grp = gb + b;
-            if (grp >= gw1) break;
-            float s[RT][2];
-            ZeroBias<XT> zb[RT][2];
-#pragma unroll
-            for (int r = 0; r < RT; ++r)
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int64_t gi = (int64_t)nrow[r][h] * G + grp;
-                    s[r][h] = __ldg(scales + gi);
-                    zb[r][h].set(zeros ? __ldg(zeros + gi) : 8.0f);
+                for (int i = 0; i < 4; ++i) {
+                    const int n = n0 + (i < 2 ? lrow0 : lrow1);
+                    const int m = 8 * mt + 2 * t + (i & 1);
+                    if (n < N && m < M) store_out<XT>(Y, (int64_t)m * N + n, acc[mt][i]);
                 }
-            float part[RT][MT][4];
+            return;
+        }
+        // partial: slot 0 for the CTA's first row block, 1 for its last
+        const int slot = 2 * c + (rb == u0 / wk.KS ? 0 : 1);
+        float *dst = partial + (int64_t)slot * kUnitRows * M;
 #pragma unroll
-            for (int r = 0; r < RT; ++r)
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                for (int mt = 0; mt < MT; ++mt)
+            for (int i = 0; i < 4; ++i) {
+                const int r = i < 2 ? lrow0 : lrow1;
+                const int m = 8 * mt + 2 * t + (i & 1);
+                if (m < M) dst[r * M + m] = acc[mt][i];
+            }
+        __threadfence();
+        __syncwarp();
+        const int cf = owner(wk, rb * wk.KS), cl = owner(wk, (rb + 1) * wk.KS - 1);
+        unsigned *cnt = counters + rb * kConsumerWarps + warp;
+        unsigned prev = 0;
+        if (lane == 0) prev = atomicAdd(cnt, 1u);
+        prev = __shfl_sync(0xffffffffu, prev, 0);
+        if (prev != (unsigned)(cl - cf)) return;
+        __threadfence();
+        for (int e = lane; e < 16 * M; e += 32) {
+            const int r = 16 * warp + (e & 15), m = e >> 4;
+            const int n = n0 + r;
+            if (n >= N) continue;
+            float v = 0.0f;
+            for (int cc = cf; cc <= cl; ++cc) {
+                const int sl = 2 * cc + (rb == range_start(wk, cc) / wk.KS ? 0 : 1);
+                v += __ldcg(partial + ((int64_t)sl * kUnitRows + r) * M + m);
+            }
+            store_out<XT>(Y, (int64_t)m * N + n, v);
+        }
+        __syncwarp();
+        if (lane == 0) *cnt = 0u;  // re-arm for the next call
+    };
+
+    for (int u = u0; u < u1; ++u) {
+        const int it = u - u0;
+        const int s = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        const int rb = u / wk.KS, ks = u % wk.KS;
+        if (rb != cur_rb) {
+            if (cur_rb >= 0) flush(cur_rb);
+            cur_rb = rb;
+            first_ks = ks;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) part[r][mt][i] = 0.0f;
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[mt][i] = 0.0f;
+        }
+        last_ks = ks;
+        const int ng = min(2, G - 2 * ks);  // groups in this unit
+        // scales and zero points of this thread's rows (clamped past N)
+        const int n_a = min(rb * kUnitRows + lrow0, N - 1);
+        const int n_b = min(rb * kUnitRows + lrow1, N - 1);
+        float sa[2], sb[2], za[2], zbv[2];
+#pragma unroll
+        for (int gi = 0; gi < 2; ++gi) {
+            const int grp = min(2 * ks + gi, G - 1);
+            sa[gi] = __ldg(scales + (int64_t)n_a * G + grp);
+            sb[gi] = __ldg(scales + (int64_t)n_b * G + grp);
+            za[gi] = zeros ? __ldg(zeros + (int64_t)n_a * G + grp) : 8.0f;
+            zbv[gi] = zeros ? __ldg(zeros + (int64_t)n_b * G + grp) : 8.0f;
+        }
+        const bool got = __all_sync(0xffffffffu,
+                                    mbar_wait(smem_u32(&sh->full[s]), ph, abort_flag, status));
+        if (!got) { ok = false; break; }
+        const uint8_t *unit = ring + s * kUnitBytes;
+#pragma unroll
+        for (int gi = 0; gi < 2; ++gi) {
+            if (gi >= ng) break;
+            const int chunk = (4 * gi + t) ^ swz;
+            const uint4 wa = *reinterpret_cast<const uint4 *>(unit + lrow0 * 128 + chunk * 16);
+            const uint4 wb = *reinterpret_cast<const uint4 *>(unit + lrow1 * 128 + chunk * 16);
+            uint32_t zba, zqa, zbb, zqb;
+            zero_bias<XT>(za[gi], zba, zqa);
+            zero_bias<XT>(zbv[gi], zbb, zqb);
+            const int kx = (2 * ks + gi) * kGroup;
+            float part[MT][4];
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) part[mt][i] = 0.0f;
+            const uint32_t wav[4] = {wa.x, wa.y, wa.z, wa.w};
+            const uint32_t wbv[4] = {wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 uint4 xv[MT];
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt) {
                     xv[mt] = make_uint4(0, 0, 0, 0);
-                    if (xval[mt]) xv[mt] = ldg_keep(xrow[mt] + grp * kGroup + 8 * j);
+                    if (xval[mt]) xv[mt] = __ldg(reinterpret_cast<const uint4 *>(xrow[mt] + kx + 8 * j));
                 }
-#pragma unroll
-                for (int r = 0; r < RT; ++r) {
-                    uint32_t pa[4], pb[4];  // rows g and g+8
-                    const uint32_t wa = j == 0 ? wv[b][r][0].x : j == 1 ? wv[b][r][0].y
-                                      : j == 2 ? wv[b][r][0].z : wv[b][r][0].w;
-                    const uint32_t wbw = j == 0 ? wv[b][r][1].x : j == 1 ? wv[b][r][1].y
-                                       : j == 2 ? wv[b][r][1].z : wv[b][r][1].w;
-                    dequant_word<XT>(wa, zb[r][0], pa);
-                    dequant_word<XT>(wbw, zb[r][1], pb);
-                    const uint32_t a0[4] = {pa[0], pb[0], pa[1], pb[1]};
-                    const uint32_t a1[4] = {pa[2], pb[2], pa[3], pb[3]};
-#pragma unroll
-                    for (int mt = 0; mt < MT; ++mt) {
-                        mma16816<XT>(part[r][mt], a0, xv[mt].x, xv[mt].y);
-                        mma16816<XT>(part[r][mt], a1, xv[mt].z, xv[mt].w);
-                    }
-                }
-            }
-#pragma unroll
-            for (int r = 0; r < RT; ++r)
+                uint32_t pa[4], pb[4];
+                dequant_word<XT>(wav[j], zba, zqa, pa);
+                dequant_word<XT>(wbv[j], zbb, zqb, pb);
+                const uint32_t a0[4] = {pa[0], pb[0], pa[1], pb[1]};
+                const uint32_t a1[4] = {pa[2], pb[2], pa[3], pb[3]};
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt) {
-                    acc[r][mt][0] = fmaf(s[r][0], part[r][mt][0], acc[r][mt][0]);
-                    acc[r][mt][1] = fmaf(s[r][0], part[r][mt][1], acc[r][mt][1]);
-                    acc[r][mt][2] = fmaf(s[r][1], part[r][mt][2], acc[r][mt][2]);
-                    acc[r][mt][3] = fmaf(s[r][1], part[r][mt][3], acc[r][mt][3]);
+                    mma16816<XT>(part[mt], a0, xv[mt].x, xv[mt].y);
+                    mma16816<XT>(part[mt], a1, xv[mt].z, xv[mt].w);
                 }
-        }
-    }
-
-    // ---- reduce the WK warps of each row tile in fixed order ----
-#pragma unroll
-    for (int r = 0; r < RT; ++r)
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int row = wn * 16 * RT + 16 * r + g + 8 * (i >> 1);
-                const int m = 8 * mt + 2 * t + (i & 1);
-                red[wk][row][m] = acc[r][mt][i];
             }
-    __syncthreads();
-
-    const int Mv = M < MP ? M : MP;
-    if (splits == 1) {
-        for (int e = threadIdx.x; e < ROWS * Mv; e += kThreads) {
-            const int row = e % ROWS, m = e / ROWS;
-            const int n = n_cta + row;
-            if (n >= N) continue;
-            float v = 0.0f;
 #pragma unroll
-            for (int w = 0; w < WK; ++w) v += red[w][row][m];
-            store_out<XT>(Y, (int64_t)m * N + n, v);
+            for (int mt = 0; mt < MT; ++mt) {
+                acc[mt][0] = fmaf(sa[gi], part[mt][0], acc[mt][0]);
+                acc[mt][1] = fmaf(sa[gi], part[mt][1], acc[mt][1]);
+                acc[mt][2] = fmaf(sb[gi], part[mt][2], acc[mt][2]);
+                acc[mt][3] = fmaf(sb[gi], part[mt][3], acc[mt][3]);
+            }
         }
-        return;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sh->empty[s]));
     }
-
-    // ---- split-K across CTAs: partial to workspace, last CTA finishes ----
-    for (int e = threadIdx.x; e < ROWS * Mv; e += kThreads) {
-        const int row = e % ROWS, m = e / ROWS;
-        const int n = n_cta + row;
-        if (n >= N) continue;
-        float v = 0.0f;
-#pragma unroll
-        for (int w = 0; w < WK; ++w) v += red[w][row][m];
-        ws_partial[((int64_t)split * M + m) * N + n] = v;
-    }
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const unsigned prev = atomicAdd(ws_count + rb, 1u);
-        s_last = (prev == (unsigned)(splits - 1)) ? 1u : 0u;
-    }
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    for (int e = threadIdx.x; e < ROWS * Mv; e += kThreads) {
-        const int row = e % ROWS, m = e / ROWS;
-        const int n = n_cta + row;
-        if (n >= N) continue;
-        float v = 0.0f;
-        for (int sp = 0; sp < splits; ++sp) v += __ldcg(ws_partial + ((int64_t)sp * M + m) * N + n);
-        store_out<XT>(Y, (int64_t)m * N + n, v);
-    }
-    if (threadIdx.x == 0) ws_count[rb] = 0u;  // re-arm for the next call
+    if (ok && cur_rb >= 0) flush(cur_rb);
 }
 
-DecodeCfg pick_cfg(int64_t M) {
-    if (M <= 8) return {1, 1, 1};
-    if (M <= 16) return {2, 1, 2};
-    if (M <= 24) return {3, 2, 2};
-    return {4, 2, 4};
-}
+// ---- host side --------------------------------------------------------------------------
 
-struct Plan {
-    DecodeCfg c;
-    int row_blocks, splits;
-    size_t partial_bytes, count_bytes;
-};
+int mt_for(int64_t M) { return (int)((M + 7) / 8); }
 
-int make_plan(int64_t M, int64_t K, int64_t N, Plan *p) {
+int make_work(int64_t M, int64_t K, int64_t N, Work *w, size_t *ws_bytes) {
     DeviceInfo di;
     int st = device_info(&di);
     if (st != W4_OK) return st;
-    p->c = pick_cfg(M);
-    const int rows = rows_per_cta(p->c.RT, p->c.WN);
-    p->row_blocks = (int)((N + rows - 1) / rows);
-    const int G = (int)(K / kGroup);
-    const int WK = kWarps / p->c.WN;
-    // enough CTAs for ~2 per SM, keeping >= 2 groups per warp
-    int want = (2 * di.sm_count + p->row_blocks - 1) / p->row_blocks;
-    int maxs = G / (2 * WK);
-    if (maxs < 1) maxs = 1;
-    if (want > maxs) want = maxs;
-    if (want > 16) want = 16;
-    p->splits = want < 1 ? 1 : want;
-    if (p->row_blocks > kMaxCounters) p->splits = 1;
-    if (p->splits > 1) {
-        p->partial_bytes = ((size_t)p->splits * M * N * sizeof(float) + 255) & ~(size_t)255;
-        p->count_bytes = kCounterBytes;
-    } else {
-        p->partial_bytes = p->count_bytes = 0;
-    }
+    w->G = (int)(K / kGroup);
+    w->KS = (int)((K + kUnitK - 1) / kUnitK);
+    w->RB = (int)((N + kUnitRows - 1) / kUnitRows);
+    w->U = w->KS * w->RB;
+    w->P = w->U < di.sm_count ? w->U : di.sm_count;
+    // many row blocks per CTA (or too many for the counter area): whole row blocks
+    w->aligned = (w->RB >= 8 * w->P || w->RB > kMaxRowBlocks) ? 1 : 0;
+    if (w->aligned && w->P > w->RB) w->P = w->RB;
+    *ws_bytes = w->aligned ? 0 : kCounterBytes + (size_t)2 * w->P * kUnitRows * M * sizeof(float);
     return W4_OK;
 }
 
-template <int XT, int MT, int RT, int WN>
-int launch_t(const Plan &p, const void *X, int64_t M, const uint8_t *packed, const float *scales,
+template <int XT, int MT>
+int launch_t(const Work &w, const CUtensorMap &map, const void *X, int64_t M, const float *scales,
              const float *zeros, int64_t K, int64_t N, void *Y, void *ws, cudaStream_t stream) {
-    float *partial = nullptr;
-    unsigned *count = nullptr;
-    if (p.splits > 1) {
-        count = static_cast<unsigned *>(ws);
-        partial = reinterpret_cast<float *>(static_cast<char *>(ws) + p.count_bytes);
+    auto kern = decode_kernel<XT, MT>;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return set_error(W4_ERR_CUDA, "cudaGetDevice", nullptr);
+    static bool attr_done[64] = {};
+    if (!attr_done[dev]) {
+        cudaError_t e =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(decode smem)", e);
+        attr_done[dev] = true;
     }
-    dim3 grid(p.row_blocks, p.splits);
-    decode_kernel<XT, MT, RT, WN><<<grid, kThreads, 0, stream>>>(
-        static_cast<const uint16_t *>(X), (int)M, reinterpret_cast<const uint32_t *>(packed),
-        scales, zeros, (int)K, (int)N, Y, partial, count, p.splits);
+    unsigned *status = device_status_ptr();
+    if (!status) return W4_ERR_CUDA;
+    unsigned *counters = nullptr;
+    float *partial = nullptr;
+    if (!w.aligned) {
+        counters = static_cast<unsigned *>(ws);
+        partial = reinterpret_cast<float *>(static_cast<char *>(ws) + kCounterBytes);
+    }
+    kern<<<w.P, kThreads, kSmemBytes, stream>>>(map, static_cast<const uint16_t *>(X), (int)M, scales,
+                                                zeros, (int)K, (int)N, Y, counters, partial, w, status);
     return cuda_status(cudaGetLastError());
 }
 
 template <int XT>
-int launch_x(const Plan &p, const void *X, int64_t M, const uint8_t *packed, const float *scales,
+int launch_x(const Work &w, const CUtensorMap &map, const void *X, int64_t M, const float *scales,
              const float *zeros, int64_t K, int64_t N, void *Y, void *ws, cudaStream_t s) {
-    switch (p.c.MT) {
-        case 1: return launch_t<XT, 1, 1, 1>(p, X, M, packed, scales, zeros, K, N, Y, ws, s);
-        case 2: return launch_t<XT, 2, 1, 2>(p, X, M, packed, scales, zeros, K, N, Y, ws, s);
-        case 3: return launch_t<XT, 3, 2, 2>(p, X, M, packed, scales, zeros, K, N, Y, ws, s);
-        default: return launch_t<XT, 4, 2, 4>(p, X, M, packed, scales, zeros, K, N, Y, ws, s);
+    switch (mt_for(M)) {
+        case 1: return launch_t<XT, 1>(w, map, X, M, scales, zeros, K, N, Y, ws, s);
+        case 2: return launch_t<XT, 2>(w, map, X, M, scales, zeros, K, N, Y, ws, s);
+        case 3: return launch_t<XT, 3>(w, map, X, M, scales, zeros, K, N, Y, ws, s);
+        default: return launch_t<XT, 4>(w, map, X, M, scales, zeros, K, N, Y, ws, s);
     }
 }
 
 }  // namespace
 
+size_t decode_counter_bytes() { return kCounterBytes; }
+
 size_t decode_workspace_bytes(int64_t M, int64_t K, int64_t N, int group) {
     (void)group;
-    Plan p;
-    if (make_plan(M, K, N, &p) != W4_OK) return 0;
-    return p.partial_bytes + p.count_bytes;
+    Work w;
+    size_t b = 0;
+    if (make_work(M, K, N, &w, &b) != W4_OK) return 0;
+    return b;
 }
 
 int launch_decode(const void *X, int xt, int64_t M, const uint8_t *packed, const float *scales,
                   const float *zeros, int64_t K, int64_t N, void *Y, void *workspace,
                   size_t workspace_bytes, cudaStream_t stream) {
-    Plan p;
-    int st = make_plan(M, K, N, &p);
+    Work w;
+    size_t need = 0;
+    int st = make_work(M, K, N, &w, &need);
     if (st != W4_OK) return st;
-    if (p.partial_bytes + p.count_bytes > workspace_bytes) return W4_ERR_INVALID_ARG;
+    if (need > workspace_bytes || (need > 0 && !workspace))
+        return set_error(W4_ERR_INVALID_ARG, "w4a16_gemm", "workspace smaller than needed");
+    CUtensorMap map;
+    if ((st = make_map_2d(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)K / 2, (uint64_t)N,
+                          (uint64_t)K / 2, kUnitK / 2, kUnitRows, CU_TENSOR_MAP_SWIZZLE_128B,
+                          "tensor map of packed (decode)")) != W4_OK)
+        return st;
     if (xt == W4_F16)
-        return launch_x<W4_F16>(p, X, M, packed, scales, zeros, K, N, Y, workspace, stream);
-    return launch_x<W4_BF16>(p, X, M, packed, scales, zeros, K, N, Y, workspace, stream);
+        return launch_x<W4_F16>(w, map, X, M, scales, zeros, K, N, Y, workspace, stream);
+    return launch_x<W4_BF16>(w, map, X, M, scales, zeros, K, N, Y, workspace, stream);
 }
 
 }  // namespace w4

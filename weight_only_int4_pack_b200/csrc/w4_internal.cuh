@@ -3,6 +3,8 @@
 // part of the public ABI (that is include/w4a16.h).
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -30,6 +32,15 @@ int cuda_fail(const char *what, cudaError_t e);  // W4_ERR_CUDA with the runtime
 
 inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? W4_OK : cuda_fail("kernel launch", e); }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (the
+// library does not link libcuda); records an error and returns null if absent.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
+// Encodes a 2-D tiled tensor map; W4_OK or W4_ERR_CUDA (with a message).
+int make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *ptr, uint64_t inner,
+                uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                CUtensorMapSwizzle swz, const char *what);
+
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // ---- launchers (one per translation unit) ----
@@ -39,6 +50,7 @@ int launch_quantize(const void *W, int wt, int64_t K, int64_t N, int group, int 
 
 // decode path, M <= 32
 size_t decode_workspace_bytes(int64_t M, int64_t K, int64_t N, int group);
+size_t decode_counter_bytes();  // leading workspace bytes that must read as zero
 int launch_decode(const void *X, int xt, int64_t M, const uint8_t *packed, const float *scales,
                   const float *zeros, int64_t K, int64_t N, void *Y, void *workspace,
                   size_t workspace_bytes, cudaStream_t stream);

@@ -28,9 +28,6 @@
 namespace {
 
 constexpr size_t kScratchBytes = size_t(4) << 20;  // 4 MiB per device
-// Start of the workspace that must read as zero before a launch: the decode
-// kernel's arrival counters live in the first 4 KiB.
-constexpr size_t kZeroedBytes = 4096;
 
 __device__ __align__(256) unsigned char g_w4_scratch[kScratchBytes];
 
@@ -91,7 +88,8 @@ extern "C" int w4a16_gemm_noalloc(const void *X, int xt, int64_t M, const uint8_
         ws_bytes = kScratchBytes;
         // The array keeps whatever the previous call left; the counters must
         // start at zero.
-        cudaError_t e = cudaMemsetAsync(ws, 0, need < kZeroedBytes ? need : kZeroedBytes, s);
+        const size_t zeroed = w4::decode_counter_bytes();
+        cudaError_t e = cudaMemsetAsync(ws, 0, need < zeroed ? need : zeroed, s);
         if (e != cudaSuccess) return w4::cuda_fail("cudaMemsetAsync(scratch counters)", e);
     }
     return w4::launch_decode(X, xt, M, packed, scales, zeros, K, N, Y, ws, ws_bytes, s);

@@ -41,14 +41,11 @@
 // wait (bounded) for their copies / MMAs in flight, and TMEM is freed before
 // the CTA exits.
 
-#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
-#include <cudaTypedefs.h>
 
 #include <stdio.h>
 
-#include <mutex>
 
 #include "w4_internal.cuh"
 
@@ -510,40 +507,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
 }
 
 // ---- host side --------------------------------------------------------------------------
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
-                                             &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-int make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *ptr, uint64_t inner,
-                uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
-                CUtensorMapSwizzle swz, const char *what) {
-    auto fn = encode_fn();
-    if (!fn) return set_error(W4_ERR_CUDA, what, "cuTensorMapEncodeTiled entry point not found");
-    cuuint64_t dims[2] = {inner, outer};
-    cuuint64_t strides[1] = {row_bytes};
-    cuuint32_t box[2] = {box_inner, box_outer};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(map, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) {
-        char buf[64];
-        snprintf(buf, sizeof buf, "cuTensorMapEncodeTiled returned CUresult %d", (int)r);
-        return set_error(W4_ERR_CUDA, what, buf);
-    }
-    return W4_OK;
-}
 
 template <int XT>
 int launch_t(const void *X, int64_t M, const uint8_t *packed, const float *scales,

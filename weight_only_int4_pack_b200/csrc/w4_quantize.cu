@@ -110,7 +110,7 @@ __device__ __forceinline__ bool codes_fast(const float w[8], float r, float zp, 
 
 // The plain definition with correctly rounded division (rare path).
 template <bool SYM>
-__device__ __noinline__ void codes_exact(const float w[8], float s, float zp, uint32_t bits[8]) {
+__device__ __forceinline__ void codes_exact(const float w[8], float s, float zp, uint32_t bits[8]) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const float a = __fdiv_rn(w[j], s);
