@@ -54,11 +54,9 @@ constexpr int kGroup = 128;
 constexpr int kUnitRows = 128;                  // weight rows per unit
 constexpr int kUnitK = 256;                     // k per unit (two groups, 128 bytes of codes per row)
 constexpr int kUnitBytes = kUnitRows * kUnitK / 2;  // 16 KB
-constexpr int kStages = 8;
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = 32 * kConsumerWarps;    // 256
 constexpr int kThreads = kConsumers + 32;          // + producer warp
-constexpr int kSmemBytes = kStages * kUnitBytes + 1024 + 256;
 // Workspace: arrival counters (one per row block and consumer warp) first,
 // then two partial slots per CTA ([2 * ctas][128 rows][M] fp32).  The counter
 // area is fixed so that one workspace serves calls of any shape; row-block
@@ -194,9 +192,20 @@ __device__ __forceinline__ void store_out(void *Y, int64_t idx, float v) {
         reinterpret_cast<__nv_bfloat16 *>(Y)[idx] = __float2bfloat16_rn(v);
 }
 
+// Stage layout for MT n8-tiles of X: the unit's codes (128 rows x 128 B),
+// then X[0 .. 8*MT)[k0 .. k0+256) as four 64-k boxes of 8*MT rows x 128 B,
+// all with the 128-byte swizzle (TMA zero-fills rows >= M and k >= K).
+template <int MT>
+struct StageCfg {
+    static constexpr int kXBox = 8 * MT * 128;                  // one 64-k box of X
+    static constexpr int kBytes = kUnitBytes + 4 * kXBox;        // 20..32 KB
+    static constexpr int kStages = (196 * 1024) / kBytes < 8 ? (196 * 1024) / kBytes : 8;
+    static constexpr int kSmem = kStages * kBytes + 1024 + 256;
+};
+
 struct Shared {
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
+    uint64_t full[8];
+    uint64_t empty[8];
     int abort_flag;
 };
 
@@ -221,14 +230,16 @@ __device__ __forceinline__ int owner(const Work &w, int u) {
 
 template <int XT, int MT>
 __global__ void __launch_bounds__(kThreads, 1)
-decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__restrict__ X, int M,
-              const float *__restrict__ scales, const float *__restrict__ zeros, int K, int N,
+decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+              int M, const float *__restrict__ scales, const float *__restrict__ zeros, int K, int N,
               void *__restrict__ Y, unsigned *__restrict__ counters, float *__restrict__ partial,
               const Work wk, unsigned *__restrict__ status) {
+    using SC = StageCfg<MT>;
+    constexpr int S = SC::kStages;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
-    Shared *sh = reinterpret_cast<Shared *>(ring + kStages * kUnitBytes);
+    Shared *sh = reinterpret_cast<Shared *>(ring + S * SC::kBytes);
     volatile int *abort_flag = &sh->abort_flag;
 
     const int warp = threadIdx.x >> 5;
@@ -238,7 +249,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__rest
     const int u1 = range_start(wk, c + 1);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < S; ++s) {
             mbar_init(smem_u32(&sh->full[s]), 1);
             mbar_init(smem_u32(&sh->empty[s]), kConsumerWarps);
         }
@@ -253,25 +264,29 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__rest
             int u = u0;
             for (; u < u1; ++u) {
                 const int it = u - u0;
-                const int s = it % kStages;
-                const uint32_t ph = (it / kStages) & 1;
+                const int s = it % S;
+                const uint32_t ph = (it / S) & 1;
                 if (!mbar_wait(smem_u32(&sh->empty[s]), ph ^ 1, abort_flag, status)) break;
                 const uint32_t fb = smem_u32(&sh->full[s]);
-                mbar_arrive_tx(fb, kUnitBytes);
+                mbar_arrive_tx(fb, SC::kBytes);
                 const int rb = u / wk.KS, ks = u % wk.KS;
-                tma_load_2d(smem_u32(ring + s * kUnitBytes), &tmap_w, ks * (kUnitK / 2),
-                            rb * kUnitRows, fb);
+                uint8_t *st = ring + s * SC::kBytes;
+                tma_load_2d(smem_u32(st), &tmap_w, ks * (kUnitK / 2), rb * kUnitRows, fb);
+#pragma unroll
+                for (int b = 0; b < 4; ++b)
+                    tma_load_2d(smem_u32(st + kUnitBytes + b * SC::kXBox), &tmap_x,
+                                ks * kUnitK + 64 * b, 0, fb);
             }
             // wait (bounded) for the copies still in flight before the CTA may exit
-            for (int j = (u - u0 > kStages ? u - u0 - kStages : 0); j < u - u0; ++j) {
+            for (int j = (u - u0 > S ? u - u0 - S : 0); j < u - u0; ++j) {
                 const unsigned long long t0 = globaltimer();
-                while (!mbar_try(smem_u32(&sh->full[j % kStages]), (j / kStages) & 1) &&
+                while (!mbar_try(smem_u32(&sh->full[j % S]), (j / S) & 1) &&
                        globaltimer() - t0 < kWaitNs) {
                 }
             }
         }
         __syncwarp();
-        return;  // the producer takes no part in the consumers' named barriers
+        return;
     }
 
     // ---------------- consumers ----------------
@@ -281,16 +296,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__rest
     const int lrow1 = lrow0 + 8;
     const int swz = lrow0 & 7;                   // swizzle key of both rows
     const int G = wk.G;
-
-    // X rows of this thread's B fragments (rows >= M give zero columns)
-    const uint16_t *xrow[MT];
-    bool xval[MT];
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-        const int m = 8 * mt + g;
-        xval[mt] = m < M;
-        xrow[mt] = X + (int64_t)(xval[mt] ? m : 0) * K + 32 * t;
-    }
 
     float acc[MT][4];
     int cur_rb = -1, first_ks = 0, last_ks = -1;
@@ -347,10 +352,27 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__rest
         if (lane == 0) *cnt = 0u;  // re-arm for the next call
     };
 
+    // scales and zero points of one unit for this thread's two rows
+    float sa[2], sb[2], za[2], zbv[2];
+    auto load_sz = [&](int u) {
+        const int rb = u / wk.KS, ks = u % wk.KS;
+        const int n_a = min(rb * kUnitRows + lrow0, N - 1);
+        const int n_b = min(rb * kUnitRows + lrow1, N - 1);
+#pragma unroll
+        for (int gi = 0; gi < 2; ++gi) {
+            const int grp = min(2 * ks + gi, G - 1);
+            sa[gi] = __ldg(scales + (int64_t)n_a * G + grp);
+            sb[gi] = __ldg(scales + (int64_t)n_b * G + grp);
+            za[gi] = zeros ? __ldg(zeros + (int64_t)n_a * G + grp) : 8.0f;
+            zbv[gi] = zeros ? __ldg(zeros + (int64_t)n_b * G + grp) : 8.0f;
+        }
+    };
+    if (u0 < u1) load_sz(u0);
+
     for (int u = u0; u < u1; ++u) {
         const int it = u - u0;
-        const int s = it % kStages;
-        const uint32_t ph = (it / kStages) & 1;
+        const int s = it % S;
+        const uint32_t ph = (it / S) & 1;
         const int rb = u / wk.KS, ks = u % wk.KS;
         if (rb != cur_rb) {
             if (cur_rb >= 0) flush(cur_rb);
@@ -363,22 +385,16 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__rest
         }
         last_ks = ks;
         const int ng = min(2, G - 2 * ks);  // groups in this unit
-        // scales and zero points of this thread's rows (clamped past N)
-        const int n_a = min(rb * kUnitRows + lrow0, N - 1);
-        const int n_b = min(rb * kUnitRows + lrow1, N - 1);
-        float sa[2], sb[2], za[2], zbv[2];
-#pragma unroll
-        for (int gi = 0; gi < 2; ++gi) {
-            const int grp = min(2 * ks + gi, G - 1);
-            sa[gi] = __ldg(scales + (int64_t)n_a * G + grp);
-            sb[gi] = __ldg(scales + (int64_t)n_b * G + grp);
-            za[gi] = zeros ? __ldg(zeros + (int64_t)n_a * G + grp) : 8.0f;
-            zbv[gi] = zeros ? __ldg(zeros + (int64_t)n_b * G + grp) : 8.0f;
-        }
+        // this unit's scales and zero points; the next unit's are fetched
+        // while this one is computed
+        const float csa[2] = {sa[0], sa[1]}, csb[2] = {sb[0], sb[1]};
+        const float cza[2] = {za[0], za[1]}, czb[2] = {zbv[0], zbv[1]};
+        if (u + 1 < u1) load_sz(u + 1);
         const bool got = __all_sync(0xffffffffu,
                                     mbar_wait(smem_u32(&sh->full[s]), ph, abort_flag, status));
         if (!got) { ok = false; break; }
-        const uint8_t *unit = ring + s * kUnitBytes;
+        const uint8_t *unit = ring + s * SC::kBytes;
+        const uint8_t *xs = unit + kUnitBytes;
 #pragma unroll
         for (int gi = 0; gi < 2; ++gi) {
             if (gi >= ng) break;
@@ -386,9 +402,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__rest
             const uint4 wa = *reinterpret_cast<const uint4 *>(unit + lrow0 * 128 + chunk * 16);
             const uint4 wb = *reinterpret_cast<const uint4 *>(unit + lrow1 * 128 + chunk * 16);
             uint32_t zba, zqa, zbb, zqb;
-            zero_bias<XT>(za[gi], zba, zqa);
-            zero_bias<XT>(zbv[gi], zbb, zqb);
-            const int kx = (2 * ks + gi) * kGroup;
+            zero_bias<XT>(cza[gi], zba, zqa);
+            zero_bias<XT>(czb[gi], zbb, zqb);
             float part[MT][4];
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt)
@@ -396,13 +411,16 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__rest
                 for (int i = 0; i < 4; ++i) part[mt][i] = 0.0f;
             const uint32_t wav[4] = {wa.x, wa.y, wa.z, wa.w};
             const uint32_t wbv[4] = {wb.x, wb.y, wb.z, wb.w};
+            // X of k = 128 gi + 32 t + 8 j: box 2 gi + t/2, 16-byte chunk 4 (t&1) + j
+            const uint8_t *xbox = xs + (2 * gi + (t >> 1)) * SC::kXBox;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 uint4 xv[MT];
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt) {
-                    xv[mt] = make_uint4(0, 0, 0, 0);
-                    if (xval[mt]) xv[mt] = __ldg(reinterpret_cast<const uint4 *>(xrow[mt] + kx + 8 * j));
+                    const int xr = 8 * mt + g;  // row of X in the box; swizzle key xr & 7 = g
+                    xv[mt] = *reinterpret_cast<const uint4 *>(xbox + xr * 128 +
+                                                              (((4 * (t & 1) + j) ^ g) << 4));
                 }
                 uint32_t pa[4], pb[4];
                 dequant_word<XT>(wav[j], zba, zqa, pa);
@@ -417,10 +435,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__rest
             }
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
-                acc[mt][0] = fmaf(sa[gi], part[mt][0], acc[mt][0]);
-                acc[mt][1] = fmaf(sa[gi], part[mt][1], acc[mt][1]);
-                acc[mt][2] = fmaf(sb[gi], part[mt][2], acc[mt][2]);
-                acc[mt][3] = fmaf(sb[gi], part[mt][3], acc[mt][3]);
+                acc[mt][0] = fmaf(csa[gi], part[mt][0], acc[mt][0]);
+                acc[mt][1] = fmaf(csa[gi], part[mt][1], acc[mt][1]);
+                acc[mt][2] = fmaf(csb[gi], part[mt][2], acc[mt][2]);
+                acc[mt][3] = fmaf(csb[gi], part[mt][3], acc[mt][3]);
             }
         }
         __syncwarp();
@@ -450,8 +468,9 @@ int make_work(int64_t M, int64_t K, int64_t N, Work *w, size_t *ws_bytes) {
 }
 
 template <int XT, int MT>
-int launch_t(const Work &w, const CUtensorMap &map, const void *X, int64_t M, const float *scales,
+int launch_t(const Work &w, const CUtensorMap &mapw, const void *X, int64_t M, const float *scales,
              const float *zeros, int64_t K, int64_t N, void *Y, void *ws, cudaStream_t stream) {
+    using SC = StageCfg<MT>;
     auto kern = decode_kernel<XT, MT>;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
@@ -459,20 +478,25 @@ int launch_t(const Work &w, const CUtensorMap &map, const void *X, int64_t M, co
     static bool attr_done[64] = {};
     if (!attr_done[dev]) {
         cudaError_t e =
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SC::kSmem);
         if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(decode smem)", e);
         attr_done[dev] = true;
     }
     unsigned *status = device_status_ptr();
     if (!status) return W4_ERR_CUDA;
+    CUtensorMap mapx;
+    int st = make_map_2d(&mapx, CU_TENSOR_MAP_DATA_TYPE_UINT16, X, (uint64_t)K, (uint64_t)M,
+                         (uint64_t)K * 2, 64, 8 * MT, CU_TENSOR_MAP_SWIZZLE_128B,
+                         "tensor map of X (decode)");
+    if (st != W4_OK) return st;
     unsigned *counters = nullptr;
     float *partial = nullptr;
     if (!w.aligned) {
         counters = static_cast<unsigned *>(ws);
         partial = reinterpret_cast<float *>(static_cast<char *>(ws) + kCounterBytes);
     }
-    kern<<<w.P, kThreads, kSmemBytes, stream>>>(map, static_cast<const uint16_t *>(X), (int)M, scales,
-                                                zeros, (int)K, (int)N, Y, counters, partial, w, status);
+    kern<<<w.P, kThreads, SC::kSmem, stream>>>(mapw, mapx, (int)M, scales, zeros, (int)K, (int)N, Y,
+                                               counters, partial, w, status);
     return cuda_status(cudaGetLastError());
 }
 
