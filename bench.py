@@ -545,9 +545,9 @@ def run_profile_case(args):
     w4.load()
     case = args.profile
     if case.startswith("decode"):
-        if case == "decode_m1":
+        if case in ("decode_m1", "decode_m1_n4096"):
             c = synth.DECODE_M1
-            M, K, N, sym = 1, c["K"], c["Ns"][-1], c["sym"]
+            M, K, N, sym = 1, c["K"], c["Ns"][0 if case.endswith("4096") else -1], c["sym"]
         else:
             c = synth.DECODE_SMALLM
             M, K, N, sym = int(case.split("_m")[-1]), c["K"], c["N"], c["sym"]
