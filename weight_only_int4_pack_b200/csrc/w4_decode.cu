@@ -142,18 +142,18 @@ __device__ __forceinline__ void mma16816(float d[4], const uint32_t a[4], uint32
     }
 }
 
-// Biased zero point in the operand type: fp16 zb = {1024+z, 1024+z},
-// zq = {-(64+z), -(64+z)}; bf16 zb = {128+z, 128+z}.
+// Biased zero point in the operand type, built with integer ops: the zero
+// point z is an integer 0..15, and 1024 + z (fp16), 128 + z (bf16) and
+// 64 + z (fp16, mantissa step 1/16) are exact with z in the low mantissa bits.
+// fp16: zb = {1024+z, 1024+z}, zq = {-(64+z), -(64+z)}; bf16: zb = {128+z, 128+z}.
 template <int XT>
 __device__ __forceinline__ void zero_bias(float z, uint32_t &zb, uint32_t &zq) {
+    const uint32_t zi = static_cast<uint32_t>(__float2int_rn(z));
     if (XT == W4_F16) {
-        __half2 a = __float2half2_rn(1024.0f + z);
-        __half2 b = __float2half2_rn(-(64.0f + z));
-        zb = *reinterpret_cast<uint32_t *>(&a);
-        zq = *reinterpret_cast<uint32_t *>(&b);
+        zb = (0x6400u + zi) * 0x10001u;
+        zq = (0xD400u + (zi << 4)) * 0x10001u;
     } else {
-        __nv_bfloat162 a = __float2bfloat162_rn(128.0f + z);
-        zb = *reinterpret_cast<uint32_t *>(&a);
+        zb = (0x4300u + zi) * 0x10001u;
         zq = 0;
     }
 }
@@ -353,27 +353,40 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     };
 
     // scales and zero points of one unit for this thread's two rows
+    const int64_t rowoff0 = (int64_t)lrow0 * G, rowoff1 = (int64_t)lrow1 * G;
+    const int64_t blockstride = (int64_t)kUnitRows * G;
+    const int64_t lastrow = (int64_t)(N - 1) * G;
     float sa[2], sb[2], za[2], zbv[2];
-    auto load_sz = [&](int u) {
-        const int rb = u / wk.KS, ks = u % wk.KS;
-        const int n_a = min(rb * kUnitRows + lrow0, N - 1);
-        const int n_b = min(rb * kUnitRows + lrow1, N - 1);
-#pragma unroll
-        for (int gi = 0; gi < 2; ++gi) {
-            const int grp = min(2 * ks + gi, G - 1);
-            sa[gi] = __ldg(scales + (int64_t)n_a * G + grp);
-            sb[gi] = __ldg(scales + (int64_t)n_b * G + grp);
-            za[gi] = zeros ? __ldg(zeros + (int64_t)n_a * G + grp) : 8.0f;
-            zbv[gi] = zeros ? __ldg(zeros + (int64_t)n_b * G + grp) : 8.0f;
+    auto load_sz = [&](int rb, int ks) {
+        const int64_t base = rb * blockstride;
+        const int64_t ia = min(base + rowoff0, lastrow), ib = min(base + rowoff1, lastrow);
+        const int g0 = 2 * ks, g1 = min(2 * ks + 1, G - 1);
+        sa[0] = __ldg(scales + ia + g0);
+        sa[1] = __ldg(scales + ia + g1);
+        sb[0] = __ldg(scales + ib + g0);
+        sb[1] = __ldg(scales + ib + g1);
+        if (zeros) {
+            za[0] = __ldg(zeros + ia + g0);
+            za[1] = __ldg(zeros + ia + g1);
+            zbv[0] = __ldg(zeros + ib + g0);
+            zbv[1] = __ldg(zeros + ib + g1);
+        } else {
+            za[0] = za[1] = zbv[0] = zbv[1] = 8.0f;
         }
     };
-    if (u0 < u1) load_sz(u0);
+    // running (row block, k unit) of u, advanced without divisions
+    int rb = u0 / wk.KS;
+    int ks = u0 - rb * wk.KS;
+    if (u0 < u1) load_sz(rb, ks);
+    // X of k = 128 gi + 32 t + 8 j sits in box 2 gi + t/2, 16-byte chunk 4 (t&1) + j,
+    // row 8 mt + g of that box (swizzle key g)
+    const int xoff0 = (t >> 1) * SC::kXBox + g * 128;
+    const int xsw = 4 * (t & 1);
 
     for (int u = u0; u < u1; ++u) {
         const int it = u - u0;
         const int s = it % S;
         const uint32_t ph = (it / S) & 1;
-        const int rb = u / wk.KS, ks = u % wk.KS;
         if (rb != cur_rb) {
             if (cur_rb >= 0) flush(cur_rb);
             cur_rb = rb;
@@ -384,65 +397,98 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                 for (int i = 0; i < 4; ++i) acc[mt][i] = 0.0f;
         }
         last_ks = ks;
-        const int ng = min(2, G - 2 * ks);  // groups in this unit
+        const bool two = 2 * ks + 1 < G;  // this unit holds a second group
         // this unit's scales and zero points; the next unit's are fetched
         // while this one is computed
-        const float csa[2] = {sa[0], sa[1]}, csb[2] = {sb[0], sb[1]};
-        const float cza[2] = {za[0], za[1]}, czb[2] = {zbv[0], zbv[1]};
-        if (u + 1 < u1) load_sz(u + 1);
+        const float csa0 = sa[0], csa1 = sa[1], csb0 = sb[0], csb1 = sb[1];
+        uint32_t zba0, zqa0, zbb0, zqb0, zba1, zqa1, zbb1, zqb1;
+        zero_bias<XT>(za[0], zba0, zqa0);
+        zero_bias<XT>(zbv[0], zbb0, zqb0);
+        zero_bias<XT>(za[1], zba1, zqa1);
+        zero_bias<XT>(zbv[1], zbb1, zqb1);
+        int nrb = rb, nks = ks + 1;
+        if (nks == wk.KS) {
+            nks = 0;
+            ++nrb;
+        }
+        if (u + 1 < u1) load_sz(nrb, nks);
         const bool got = __all_sync(0xffffffffu,
                                     mbar_wait(smem_u32(&sh->full[s]), ph, abort_flag, status));
-        if (!got) { ok = false; break; }
+        if (!got) {
+            ok = false;
+            break;
+        }
         const uint8_t *unit = ring + s * SC::kBytes;
-        const uint8_t *xs = unit + kUnitBytes;
+        const uint8_t *xs = unit + kUnitBytes + xoff0;
+        // codes of both groups for rows a (lrow0) and b (lrow1)
+        const uint4 wa0 = *reinterpret_cast<const uint4 *>(unit + lrow0 * 128 + ((t ^ swz) << 4));
+        const uint4 wb0 = *reinterpret_cast<const uint4 *>(unit + lrow1 * 128 + ((t ^ swz) << 4));
+        const uint4 wa1 = *reinterpret_cast<const uint4 *>(unit + lrow0 * 128 + (((4 + t) ^ swz) << 4));
+        const uint4 wb1 = *reinterpret_cast<const uint4 *>(unit + lrow1 * 128 + (((4 + t) ^ swz) << 4));
+        const uint32_t wav0[4] = {wa0.x, wa0.y, wa0.z, wa0.w};
+        const uint32_t wbv0[4] = {wb0.x, wb0.y, wb0.z, wb0.w};
+        const uint32_t wav1[4] = {wa1.x, wa1.y, wa1.z, wa1.w};
+        const uint32_t wbv1[4] = {wb1.x, wb1.y, wb1.z, wb1.w};
+        // independent accumulators per n8 tile: one per (group, mma half) for
+        // MT <= 2; for larger MT the n8 tiles already give independent chains
+        constexpr bool kSplit = MT <= 2;
+        float p0a[MT][4], p0b[MT][4], p1a[MT][4], p1b[MT][4];
 #pragma unroll
-        for (int gi = 0; gi < 2; ++gi) {
-            if (gi >= ng) break;
-            const int chunk = (4 * gi + t) ^ swz;
-            const uint4 wa = *reinterpret_cast<const uint4 *>(unit + lrow0 * 128 + chunk * 16);
-            const uint4 wb = *reinterpret_cast<const uint4 *>(unit + lrow1 * 128 + chunk * 16);
-            uint32_t zba, zqa, zbb, zqb;
-            zero_bias<XT>(cza[gi], zba, zqa);
-            zero_bias<XT>(czb[gi], zbb, zqb);
-            float part[MT][4];
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                p0a[mt][i] = p1a[mt][i] = 0.0f;
+                if (kSplit) p0b[mt][i] = p1b[mt][i] = 0.0f;
+            }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint4 x0[MT], x1[MT];
+            const int ch = ((xsw + j) ^ g) << 4;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                x0[mt] = *reinterpret_cast<const uint4 *>(xs + mt * 1024 + ch);
+                x1[mt] = *reinterpret_cast<const uint4 *>(xs + 2 * SC::kXBox + mt * 1024 + ch);
+            }
+            uint32_t pa[4], pb[4], qa[4], qb[4];
+            dequant_word<XT>(wav0[j], zba0, zqa0, pa);
+            dequant_word<XT>(wbv0[j], zbb0, zqb0, pb);
+            dequant_word<XT>(wav1[j], zba1, zqa1, qa);
+            dequant_word<XT>(wbv1[j], zbb1, zqb1, qb);
+            const uint32_t a00[4] = {pa[0], pb[0], pa[1], pb[1]};
+            const uint32_t a01[4] = {pa[2], pb[2], pa[3], pb[3]};
+            const uint32_t a10[4] = {qa[0], qb[0], qa[1], qb[1]};
+            const uint32_t a11[4] = {qa[2], qb[2], qa[3], qb[3]};
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                mma16816<XT>(p0a[mt], a00, x0[mt].x, x0[mt].y);
+                mma16816<XT>(kSplit ? p0b[mt] : p0a[mt], a01, x0[mt].z, x0[mt].w);
+                if (two) {
+                    mma16816<XT>(p1a[mt], a10, x1[mt].x, x1[mt].y);
+                    mma16816<XT>(kSplit ? p1b[mt] : p1a[mt], a11, x1[mt].z, x1[mt].w);
+                }
+            }
+        }
+        if (!kSplit) {
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) part[mt][i] = 0.0f;
-            const uint32_t wav[4] = {wa.x, wa.y, wa.z, wa.w};
-            const uint32_t wbv[4] = {wb.x, wb.y, wb.z, wb.w};
-            // X of k = 128 gi + 32 t + 8 j: box 2 gi + t/2, 16-byte chunk 4 (t&1) + j
-            const uint8_t *xbox = xs + (2 * gi + (t >> 1)) * SC::kXBox;
+                for (int i = 0; i < 4; ++i) p0b[mt][i] = p1b[mt][i] = 0.0f;
+        }
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                uint4 xv[MT];
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    const int xr = 8 * mt + g;  // row of X in the box; swizzle key xr & 7 = g
-                    xv[mt] = *reinterpret_cast<const uint4 *>(xbox + xr * 128 +
-                                                              (((4 * (t & 1) + j) ^ g) << 4));
-                }
-                uint32_t pa[4], pb[4];
-                dequant_word<XT>(wav[j], zba, zqa, pa);
-                dequant_word<XT>(wbv[j], zbb, zqb, pb);
-                const uint32_t a0[4] = {pa[0], pb[0], pa[1], pb[1]};
-                const uint32_t a1[4] = {pa[2], pb[2], pa[3], pb[3]};
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    mma16816<XT>(part[mt], a0, xv[mt].x, xv[mt].y);
-                    mma16816<XT>(part[mt], a1, xv[mt].z, xv[mt].w);
-                }
-            }
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-                acc[mt][0] = fmaf(csa[gi], part[mt][0], acc[mt][0]);
-                acc[mt][1] = fmaf(csa[gi], part[mt][1], acc[mt][1]);
-                acc[mt][2] = fmaf(csb[gi], part[mt][2], acc[mt][2]);
-                acc[mt][3] = fmaf(csb[gi], part[mt][3], acc[mt][3]);
-            }
+        for (int mt = 0; mt < MT; ++mt) {
+            acc[mt][0] = fmaf(csa0, p0a[mt][0] + p0b[mt][0], acc[mt][0]);
+            acc[mt][1] = fmaf(csa0, p0a[mt][1] + p0b[mt][1], acc[mt][1]);
+            acc[mt][2] = fmaf(csb0, p0a[mt][2] + p0b[mt][2], acc[mt][2]);
+            acc[mt][3] = fmaf(csb0, p0a[mt][3] + p0b[mt][3], acc[mt][3]);
+            acc[mt][0] = fmaf(csa1, p1a[mt][0] + p1b[mt][0], acc[mt][0]);
+            acc[mt][1] = fmaf(csa1, p1a[mt][1] + p1b[mt][1], acc[mt][1]);
+            acc[mt][2] = fmaf(csb1, p1a[mt][2] + p1b[mt][2], acc[mt][2]);
+            acc[mt][3] = fmaf(csb1, p1a[mt][3] + p1b[mt][3], acc[mt][3]);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sh->empty[s]));
+        rb = nrb;
+        ks = nks;
     }
     if (ok && cur_rb >= 0) flush(cur_rb);
 }
