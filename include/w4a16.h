@@ -108,9 +108,16 @@ size_t w4a16_workspace_bytes(int64_t M, int64_t K, int64_t N, int group);
  *   fp32 (the integer (u - zero) is exact in the 16-bit operand type; the
  *   group scale multiplies the fp32 partial sum of its group) and rounded
  *   once to the output dtype.
- *   M <= 32 runs the decode path (split-K tensor-core GEMV); larger M runs
- *   the tcgen05 path (TMA-staged X, dequantized W tiles in shared memory,
- *   accumulators in tensor memory).
+ *   M <= 32 runs the decode path (persistent stream-K tensor-core GEMV);
+ *   larger M runs the tcgen05 path (TMA-staged X, dequantized W tiles in
+ *   shared memory, accumulators in tensor memory).
+ *   The decode path is launched with programmatic dependent launch: it may
+ *   start while the preceding kernel of the stream finishes, and it starts
+ *   streaming `packed` before that kernel has completed (X, scales, zeros, Y
+ *   and the workspace are touched only after).  So `packed` must not be
+ *   written by the immediately preceding kernel if that kernel itself allows
+ *   early dependent launch (the kernels of this library that write `packed`
+ *   do not).
  *   workspace / workspace_bytes: at least w4a16_workspace_bytes(M, K, N, group)
  *   bytes of device memory prepared as described there (may be NULL when
  *   that size is 0); a smaller workspace returns W4_ERR_INVALID_ARG.

@@ -28,6 +28,10 @@
 //     warp to arrive on that (row block, warp) counter adds the slots in CTA
 //     order, writes Y and re-arms the counter.  No warp ever waits for
 //     another warp, and the result is deterministic.
+//   * Programmatic dependent launch: the kernel may start while the preceding
+//     kernel of the stream is finishing; the producer requests the first
+//     ring of packed codes at once and everything else (X, scales, zeros,
+//     Y, workspace) is touched only after griddepcontrol.wait.
 //   * Fragment layout: thread (g, t) holds k = 32t..32t+31 of each group, so
 //     mma (word j, half h) maps the fragment's k indices {2t,2t+1,2t+8,2t+9}
 //     to k = 32t + 8j + 4h + {0,1,2,3}; the packed layout puts consecutive k
@@ -54,15 +58,12 @@ constexpr int kGroup = 128;
 constexpr int kUnitRows = 128;                  // weight rows per unit
 constexpr int kUnitK = 256;                     // k per unit (two groups, 128 bytes of codes per row)
 constexpr int kUnitBytes = kUnitRows * kUnitK / 2;  // 16 KB
-constexpr int kConsumerWarps = 8;
-constexpr int kConsumers = 32 * kConsumerWarps;    // 256
-constexpr int kThreads = kConsumers + 32;          // + producer warp
 // Workspace: arrival counters (one per row block and consumer warp) first,
 // then two partial slots per CTA ([2 * ctas][128 rows][M] fp32).  The counter
 // area is fixed so that one workspace serves calls of any shape; row-block
 // counts beyond it switch to whole-row-block ranges, which need no workspace.
 constexpr int kMaxRowBlocks = 2048;
-constexpr int kMaxCounters = kMaxRowBlocks * kConsumerWarps;
+constexpr int kMaxCounters = kMaxRowBlocks * 8;  // one per (row block, 16-row tile)
 constexpr size_t kCounterBytes = kMaxCounters * sizeof(unsigned);
 constexpr unsigned long long kWaitNs = 2000000000ull;
 
@@ -192,20 +193,31 @@ __device__ __forceinline__ void store_out(void *Y, int64_t idx, float v) {
         reinterpret_cast<__nv_bfloat16 *>(Y)[idx] = __float2bfloat16_rn(v);
 }
 
-// Stage layout for MT n8-tiles of X: the unit's codes (128 rows x 128 B),
-// then X[0 .. 8*MT)[k0 .. k0+256) as four 64-k boxes of 8*MT rows x 128 B,
-// all with the 128-byte swizzle (TMA zero-fills rows >= M and k >= K).
-template <int MT>
-struct StageCfg {
-    static constexpr int kXBox = 8 * MT * 128;                  // one 64-k box of X
-    static constexpr int kBytes = kUnitBytes + 4 * kXBox;        // 20..32 KB
-    static constexpr int kStages = (196 * 1024) / kBytes < 8 ? (196 * 1024) / kBytes : 8;
-    static constexpr int kSmem = kStages * kBytes + 1024 + 256;
+// Kernel configuration for MT n8-tiles of X and CW consumer warps.
+//   CW = 8:  warp w owns unit rows 16w..16w+15 and both groups of every unit.
+//   CW = 16: warps w and w+8 own the same 16 rows; warp w + 8h takes group h
+//            of every unit, and the pair adds its two halves through shared
+//            memory when a row block ends (twice the warps per scheduler to
+//            hide the dequant/MMA latency, at small M where registers allow).
+// Stage layout: the unit's codes (128 rows x 128 B), then X[0 .. 8*MT)[k0 ..
+// k0+256) as four 64-k boxes of 8*MT rows x 128 B, all with the 128-byte
+// swizzle (TMA zero-fills rows >= M and k >= K).
+template <int MT, int CW>
+struct Cfg {
+    static constexpr int kHalves = CW / 8;
+    static constexpr int kThreads = 32 * (CW + 1);
+    static constexpr int kXBox = 8 * MT * 128;
+    static constexpr int kBytes = kUnitBytes + 4 * kXBox;  // 20..32 KB
+    static constexpr int kStages = (192 * 1024) / kBytes < 8 ? (192 * 1024) / kBytes : 8;
+    static constexpr int kXchgBytes = kHalves == 2 ? 8 * 32 * 4 * MT * 4 : 0;
+    static constexpr int kSmem = kStages * kBytes + 1024 + 512 + kXchgBytes;
 };
 
 struct Shared {
     uint64_t full[8];
     uint64_t empty[8];
+    uint64_t pair_full[8];  // CW = 16: second half of a row tile written
+    uint64_t pair_free[8];  // CW = 16: first half read it
     int abort_flag;
 };
 
@@ -228,18 +240,20 @@ __device__ __forceinline__ int owner(const Work &w, int u) {
     return (int)(((int64_t)(u + 1) * w.P - 1) / w.U);
 }
 
-template <int XT, int MT>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int XT, int MT, int CW>
+__global__ void __launch_bounds__(Cfg<MT, CW>::kThreads, 1)
 decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
               int M, const float *__restrict__ scales, const float *__restrict__ zeros, int K, int N,
               void *__restrict__ Y, unsigned *__restrict__ counters, float *__restrict__ partial,
               const Work wk, unsigned *__restrict__ status) {
-    using SC = StageCfg<MT>;
-    constexpr int S = SC::kStages;
+    using C = Cfg<MT, CW>;
+    constexpr int S = C::kStages;
+    constexpr int H = C::kHalves;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
-    Shared *sh = reinterpret_cast<Shared *>(ring + S * SC::kBytes);
+    Shared *sh = reinterpret_cast<Shared *>(ring + S * C::kBytes);
+    float *xchg = reinterpret_cast<float *>(ring + S * C::kBytes + 512);
     volatile int *abort_flag = &sh->abort_flag;
 
     const int warp = threadIdx.x >> 5;
@@ -251,30 +265,56 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(smem_u32(&sh->full[s]), 1);
-            mbar_init(smem_u32(&sh->empty[s]), kConsumerWarps);
+            mbar_init(smem_u32(&sh->empty[s]), CW);
+        }
+        for (int r = 0; r < 8; ++r) {
+            mbar_init(smem_u32(&sh->pair_full[r]), 1);
+            mbar_init(smem_u32(&sh->pair_free[r]), 1);
         }
         sh->abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
+    // let the next kernel in the stream start its prologue as SMs free up
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-    if (warp == kConsumerWarps) {
+    if (warp == CW) {
         // ---------------- producer ----------------
         if (lane == 0) {
-            int u = u0;
+            // The packed weights are inputs no earlier kernel writes: the first
+            // ring's worth of codes is requested before waiting for the
+            // preceding kernel; X (possibly its output) only after.
+            const int pre = min(S, u1 - u0);
+            for (int it = 0; it < pre; ++it) {
+                const int u = u0 + it;
+                const uint32_t fb = smem_u32(&sh->full[it]);
+                mbar_arrive_tx(fb, C::kBytes);
+                tma_load_2d(smem_u32(ring + it * C::kBytes), &tmap_w, (u % wk.KS) * (kUnitK / 2),
+                            (u / wk.KS) * kUnitRows, fb);
+            }
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            for (int it = 0; it < pre; ++it) {
+                const int u = u0 + it;
+                uint8_t *st = ring + it * C::kBytes;
+#pragma unroll
+                for (int b = 0; b < 4; ++b)
+                    tma_load_2d(smem_u32(st + kUnitBytes + b * C::kXBox), &tmap_x,
+                                (u % wk.KS) * kUnitK + 64 * b, 0, smem_u32(&sh->full[it]));
+            }
+            int u = u0 + pre;
             for (; u < u1; ++u) {
                 const int it = u - u0;
                 const int s = it % S;
                 const uint32_t ph = (it / S) & 1;
                 if (!mbar_wait(smem_u32(&sh->empty[s]), ph ^ 1, abort_flag, status)) break;
                 const uint32_t fb = smem_u32(&sh->full[s]);
-                mbar_arrive_tx(fb, SC::kBytes);
+                mbar_arrive_tx(fb, C::kBytes);
                 const int rb = u / wk.KS, ks = u % wk.KS;
-                uint8_t *st = ring + s * SC::kBytes;
+                uint8_t *st = ring + s * C::kBytes;
                 tma_load_2d(smem_u32(st), &tmap_w, ks * (kUnitK / 2), rb * kUnitRows, fb);
 #pragma unroll
                 for (int b = 0; b < 4; ++b)
-                    tma_load_2d(smem_u32(st + kUnitBytes + b * SC::kXBox), &tmap_x,
+                    tma_load_2d(smem_u32(st + kUnitBytes + b * C::kXBox), &tmap_x,
                                 ks * kUnitK + 64 * b, 0, fb);
             }
             // wait (bounded) for the copies still in flight before the CTA may exit
@@ -291,20 +331,50 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
 
     // ---------------- consumers ----------------
     const int g = lane >> 2, t = lane & 3;
+    const int tile = warp % 8;                   // 16-row tile of the unit
+    const int half = warp / 8;                   // CW = 16: which group of each unit
     const int rsel = ((g & 1) << 2) | (g >> 1);  // unit row of mma row g (conflict-free loads)
-    const int lrow0 = 16 * warp + rsel;          // this thread's two rows in the unit
+    const int lrow0 = 16 * tile + rsel;          // this thread's two rows in the unit
     const int lrow1 = lrow0 + 8;
     const int swz = lrow0 & 7;                   // swizzle key of both rows
     const int G = wk.G;
 
     float acc[MT][4];
     int cur_rb = -1, first_ks = 0, last_ks = -1;
+    uint32_t xph = 0;  // flushes done (pair exchange parity)
     bool ok = true;
 
-    // Finishes row block rb for this warp's 16 rows.  No step waits on
-    // another warp: a row block split between CTAs has one arrival counter
-    // per (row block, warp), and the last warp to arrive adds the partials.
-    auto flush = [&](int rb) {
+    // Finishes row block rb for this tile's 16 rows.  Waits are bounded; no
+    // step waits on a warp of another tile.  A row block split between CTAs
+    // has one arrival counter per (row block, tile), and the last warp to
+    // arrive adds the partials in CTA order.
+    auto flush = [&](int rb) -> bool {
+        if (H == 2) {
+            float *xc = xchg + (tile * 32 + lane) * 4 * MT;
+            if (half == 1) {
+                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sh->pair_free[tile]), xph ^ 1,
+                                                        abort_flag, status)))
+                    return false;
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) xc[4 * mt + i] = acc[mt][i];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&sh->pair_full[tile]));
+                xph ^= 1;
+                return true;
+            }
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait(smem_u32(&sh->pair_full[tile]), xph, abort_flag, status)))
+                return false;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[mt][i] += xc[4 * mt + i];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sh->pair_free[tile]));
+            xph ^= 1;
+        }
         const int n0 = rb * kUnitRows;
         if (first_ks == 0 && last_ks == wk.KS - 1) {
 #pragma unroll
@@ -315,7 +385,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                     const int m = 8 * mt + 2 * t + (i & 1);
                     if (n < N && m < M) store_out<XT>(Y, (int64_t)m * N + n, acc[mt][i]);
                 }
-            return;
+            return true;
         }
         // partial: slot 0 for the CTA's first row block, 1 for its last
         const int slot = 2 * c + (rb == u0 / wk.KS ? 0 : 1);
@@ -331,14 +401,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         __threadfence();
         __syncwarp();
         const int cf = owner(wk, rb * wk.KS), cl = owner(wk, (rb + 1) * wk.KS - 1);
-        unsigned *cnt = counters + rb * kConsumerWarps + warp;
+        unsigned *cnt = counters + rb * 8 + tile;
         unsigned prev = 0;
         if (lane == 0) prev = atomicAdd(cnt, 1u);
         prev = __shfl_sync(0xffffffffu, prev, 0);
-        if (prev != (unsigned)(cl - cf)) return;
+        if (prev != (unsigned)(cl - cf)) return true;
         __threadfence();
         for (int e = lane; e < 16 * M; e += 32) {
-            const int r = 16 * warp + (e & 15), m = e >> 4;
+            const int r = 16 * tile + (e & 15), m = e >> 4;
             const int n = n0 + r;
             if (n >= N) continue;
             float v = 0.0f;
@@ -350,9 +420,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         }
         __syncwarp();
         if (lane == 0) *cnt = 0u;  // re-arm for the next call
+        return true;
     };
 
-    // scales and zero points of one unit for this thread's two rows
+    // scales and zero points of one unit for this thread's two rows and
+    // this warp's groups
     const int64_t rowoff0 = (int64_t)lrow0 * G, rowoff1 = (int64_t)lrow1 * G;
     const int64_t blockstride = (int64_t)kUnitRows * G;
     const int64_t lastrow = (int64_t)(N - 1) * G;
@@ -360,35 +432,33 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     auto load_sz = [&](int rb, int ks) {
         const int64_t base = rb * blockstride;
         const int64_t ia = min(base + rowoff0, lastrow), ib = min(base + rowoff1, lastrow);
-        const int g0 = 2 * ks, g1 = min(2 * ks + 1, G - 1);
-        sa[0] = __ldg(scales + ia + g0);
-        sa[1] = __ldg(scales + ia + g1);
-        sb[0] = __ldg(scales + ib + g0);
-        sb[1] = __ldg(scales + ib + g1);
-        if (zeros) {
-            za[0] = __ldg(zeros + ia + g0);
-            za[1] = __ldg(zeros + ia + g1);
-            zbv[0] = __ldg(zeros + ib + g0);
-            zbv[1] = __ldg(zeros + ib + g1);
-        } else {
-            za[0] = za[1] = zbv[0] = zbv[1] = 8.0f;
+#pragma unroll
+        for (int q = 0; q < 2 / H; ++q) {
+            const int grp = min(2 * ks + (H == 2 ? half : q), G - 1);
+            sa[q] = __ldg(scales + ia + grp);
+            sb[q] = __ldg(scales + ib + grp);
+            za[q] = zeros ? __ldg(zeros + ia + grp) : 8.0f;
+            zbv[q] = zeros ? __ldg(zeros + ib + grp) : 8.0f;
         }
     };
-    // running (row block, k unit) of u, advanced without divisions
     int rb = u0 / wk.KS;
     int ks = u0 - rb * wk.KS;
+    // everything but the packed codes is read after the preceding kernel of
+    // the stream has completed
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if (u0 < u1) load_sz(rb, ks);
-    // X of k = 128 gi + 32 t + 8 j sits in box 2 gi + t/2, 16-byte chunk 4 (t&1) + j,
-    // row 8 mt + g of that box (swizzle key g)
-    const int xoff0 = (t >> 1) * SC::kXBox + g * 128;
+    // X of k = 128 gi + 32 t + 8 j sits in box 2 gi + t/2, 16-byte chunk
+    // 4 (t&1) + j, row 8 mt + g of that box (swizzle key g)
+    const int xoff0 = (t >> 1) * C::kXBox + g * 128;
     const int xsw = 4 * (t & 1);
+    constexpr bool kSplit = MT <= 2;  // two accumulators per group: more independent MMAs
 
     for (int u = u0; u < u1; ++u) {
         const int it = u - u0;
         const int s = it % S;
         const uint32_t ph = (it / S) & 1;
         if (rb != cur_rb) {
-            if (cur_rb >= 0) flush(cur_rb);
+            if (cur_rb >= 0 && !flush(cur_rb)) { ok = false; break; }
             cur_rb = rb;
             first_ks = ks;
 #pragma unroll
@@ -397,15 +467,17 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                 for (int i = 0; i < 4; ++i) acc[mt][i] = 0.0f;
         }
         last_ks = ks;
-        const bool two = 2 * ks + 1 < G;  // this unit holds a second group
         // this unit's scales and zero points; the next unit's are fetched
         // while this one is computed
-        const float csa0 = sa[0], csa1 = sa[1], csb0 = sb[0], csb1 = sb[1];
-        uint32_t zba0, zqa0, zbb0, zqb0, zba1, zqa1, zbb1, zqb1;
-        zero_bias<XT>(za[0], zba0, zqa0);
-        zero_bias<XT>(zbv[0], zbb0, zqb0);
-        zero_bias<XT>(za[1], zba1, zqa1);
-        zero_bias<XT>(zbv[1], zbb1, zqb1);
+        float cs_a[2], cs_b[2];
+        uint32_t zba[2], zqa[2], zbb[2], zqb[2];
+#pragma unroll
+        for (int q = 0; q < 2 / H; ++q) {
+            cs_a[q] = sa[q];
+            cs_b[q] = sb[q];
+            zero_bias<XT>(za[q], zba[q], zqa[q]);
+            zero_bias<XT>(zbv[q], zbb[q], zqb[q]);
+        }
         int nrb = rb, nks = ks + 1;
         if (nks == wk.KS) {
             nks = 0;
@@ -418,72 +490,52 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             ok = false;
             break;
         }
-        const uint8_t *unit = ring + s * SC::kBytes;
+        const uint8_t *unit = ring + s * C::kBytes;
         const uint8_t *xs = unit + kUnitBytes + xoff0;
-        // codes of both groups for rows a (lrow0) and b (lrow1)
-        const uint4 wa0 = *reinterpret_cast<const uint4 *>(unit + lrow0 * 128 + ((t ^ swz) << 4));
-        const uint4 wb0 = *reinterpret_cast<const uint4 *>(unit + lrow1 * 128 + ((t ^ swz) << 4));
-        const uint4 wa1 = *reinterpret_cast<const uint4 *>(unit + lrow0 * 128 + (((4 + t) ^ swz) << 4));
-        const uint4 wb1 = *reinterpret_cast<const uint4 *>(unit + lrow1 * 128 + (((4 + t) ^ swz) << 4));
-        const uint32_t wav0[4] = {wa0.x, wa0.y, wa0.z, wa0.w};
-        const uint32_t wbv0[4] = {wb0.x, wb0.y, wb0.z, wb0.w};
-        const uint32_t wav1[4] = {wa1.x, wa1.y, wa1.z, wa1.w};
-        const uint32_t wbv1[4] = {wb1.x, wb1.y, wb1.z, wb1.w};
-        // independent accumulators per n8 tile: one per (group, mma half) for
-        // MT <= 2; for larger MT the n8 tiles already give independent chains
-        constexpr bool kSplit = MT <= 2;
-        float p0a[MT][4], p0b[MT][4], p1a[MT][4], p1b[MT][4];
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                p0a[mt][i] = p1a[mt][i] = 0.0f;
-                if (kSplit) p0b[mt][i] = p1b[mt][i] = 0.0f;
-            }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            uint4 x0[MT], x1[MT];
-            const int ch = ((xsw + j) ^ g) << 4;
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-                x0[mt] = *reinterpret_cast<const uint4 *>(xs + mt * 1024 + ch);
-                x1[mt] = *reinterpret_cast<const uint4 *>(xs + 2 * SC::kXBox + mt * 1024 + ch);
-            }
-            uint32_t pa[4], pb[4], qa[4], qb[4];
-            dequant_word<XT>(wav0[j], zba0, zqa0, pa);
-            dequant_word<XT>(wbv0[j], zbb0, zqb0, pb);
-            dequant_word<XT>(wav1[j], zba1, zqa1, qa);
-            dequant_word<XT>(wbv1[j], zbb1, zqb1, qb);
-            const uint32_t a00[4] = {pa[0], pb[0], pa[1], pb[1]};
-            const uint32_t a01[4] = {pa[2], pb[2], pa[3], pb[3]};
-            const uint32_t a10[4] = {qa[0], qb[0], qa[1], qb[1]};
-            const uint32_t a11[4] = {qa[2], qb[2], qa[3], qb[3]};
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-                mma16816<XT>(p0a[mt], a00, x0[mt].x, x0[mt].y);
-                mma16816<XT>(kSplit ? p0b[mt] : p0a[mt], a01, x0[mt].z, x0[mt].w);
-                if (two) {
-                    mma16816<XT>(p1a[mt], a10, x1[mt].x, x1[mt].y);
-                    mma16816<XT>(kSplit ? p1b[mt] : p1a[mt], a11, x1[mt].z, x1[mt].w);
-                }
-            }
-        }
-        if (!kSplit) {
+        for (int q = 0; q < 2 / H; ++q) {
+            const int gi = H == 2 ? half : q;  // group of the unit
+            if (2 * ks + gi >= G) break;       // a last unit with one group
+            const int ch0 = ((4 * gi + t) ^ swz) << 4;
+            const uint4 wa = *reinterpret_cast<const uint4 *>(unit + lrow0 * 128 + ch0);
+            const uint4 wb = *reinterpret_cast<const uint4 *>(unit + lrow1 * 128 + ch0);
+            const uint32_t wav[4] = {wa.x, wa.y, wa.z, wa.w};
+            const uint32_t wbv[4] = {wb.x, wb.y, wb.z, wb.w};
+            const uint8_t *xg = xs + 2 * gi * C::kXBox;
+            float pa_[MT][4], pb_[MT][4];
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) p0b[mt][i] = p1b[mt][i] = 0.0f;
-        }
+                for (int i = 0; i < 4; ++i) pa_[mt][i] = pb_[mt][i] = 0.0f;
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-            acc[mt][0] = fmaf(csa0, p0a[mt][0] + p0b[mt][0], acc[mt][0]);
-            acc[mt][1] = fmaf(csa0, p0a[mt][1] + p0b[mt][1], acc[mt][1]);
-            acc[mt][2] = fmaf(csb0, p0a[mt][2] + p0b[mt][2], acc[mt][2]);
-            acc[mt][3] = fmaf(csb0, p0a[mt][3] + p0b[mt][3], acc[mt][3]);
-            acc[mt][0] = fmaf(csa1, p1a[mt][0] + p1b[mt][0], acc[mt][0]);
-            acc[mt][1] = fmaf(csa1, p1a[mt][1] + p1b[mt][1], acc[mt][1]);
-            acc[mt][2] = fmaf(csb1, p1a[mt][2] + p1b[mt][2], acc[mt][2]);
-            acc[mt][3] = fmaf(csb1, p1a[mt][3] + p1b[mt][3], acc[mt][3]);
+            for (int j = 0; j < 4; ++j) {
+                uint4 xv[MT];
+                const int ch = ((xsw + j) ^ g) << 4;
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+                    xv[mt] = *reinterpret_cast<const uint4 *>(xg + mt * 1024 + ch);
+                uint32_t pa[4], pb[4];
+                dequant_word<XT>(wav[j], zba[q], zqa[q], pa);
+                dequant_word<XT>(wbv[j], zbb[q], zqb[q], pb);
+                const uint32_t a0[4] = {pa[0], pb[0], pa[1], pb[1]};
+                const uint32_t a1[4] = {pa[2], pb[2], pa[3], pb[3]};
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    mma16816<XT>(pa_[mt], a0, xv[mt].x, xv[mt].y);
+                    mma16816<XT>(kSplit ? pb_[mt] : pa_[mt], a1, xv[mt].z, xv[mt].w);
+                }
+            }
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                const float p0 = kSplit ? pa_[mt][0] + pb_[mt][0] : pa_[mt][0];
+                const float p1 = kSplit ? pa_[mt][1] + pb_[mt][1] : pa_[mt][1];
+                const float p2 = kSplit ? pa_[mt][2] + pb_[mt][2] : pa_[mt][2];
+                const float p3 = kSplit ? pa_[mt][3] + pb_[mt][3] : pa_[mt][3];
+                acc[mt][0] = fmaf(cs_a[q], p0, acc[mt][0]);
+                acc[mt][1] = fmaf(cs_a[q], p1, acc[mt][1]);
+                acc[mt][2] = fmaf(cs_b[q], p2, acc[mt][2]);
+                acc[mt][3] = fmaf(cs_b[q], p3, acc[mt][3]);
+            }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sh->empty[s]));
@@ -513,18 +565,18 @@ int make_work(int64_t M, int64_t K, int64_t N, Work *w, size_t *ws_bytes) {
     return W4_OK;
 }
 
-template <int XT, int MT>
+template <int XT, int MT, int CW>
 int launch_t(const Work &w, const CUtensorMap &mapw, const void *X, int64_t M, const float *scales,
              const float *zeros, int64_t K, int64_t N, void *Y, void *ws, cudaStream_t stream) {
-    using SC = StageCfg<MT>;
-    auto kern = decode_kernel<XT, MT>;
+    using C = Cfg<MT, CW>;
+    auto kern = decode_kernel<XT, MT, CW>;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return set_error(W4_ERR_CUDA, "cudaGetDevice", nullptr);
     static bool attr_done[64] = {};
     if (!attr_done[dev]) {
         cudaError_t e =
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SC::kSmem);
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(decode smem)", e);
         attr_done[dev] = true;
     }
@@ -541,19 +593,32 @@ int launch_t(const Work &w, const CUtensorMap &mapw, const void *X, int64_t M, c
         counters = static_cast<unsigned *>(ws);
         partial = reinterpret_cast<float *>(static_cast<char *>(ws) + kCounterBytes);
     }
-    kern<<<w.P, kThreads, SC::kSmem, stream>>>(mapw, mapx, (int)M, scales, zeros, (int)K, (int)N, Y,
-                                               counters, partial, w, status);
-    return cuda_status(cudaGetLastError());
+    // programmatic dependent launch: this kernel may start while the previous
+    // kernel of the stream finishes; it waits for it before reading X
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(w.P);
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = C::kSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mapw, mapx, (int)M, scales, zeros, (int)K, (int)N,
+                                       Y, counters, partial, w, status);
+    if (e != cudaSuccess) return cuda_fail("cudaLaunchKernelEx(decode)", e);
+    return W4_OK;
 }
 
 template <int XT>
 int launch_x(const Work &w, const CUtensorMap &map, const void *X, int64_t M, const float *scales,
              const float *zeros, int64_t K, int64_t N, void *Y, void *ws, cudaStream_t s) {
     switch (mt_for(M)) {
-        case 1: return launch_t<XT, 1>(w, map, X, M, scales, zeros, K, N, Y, ws, s);
-        case 2: return launch_t<XT, 2>(w, map, X, M, scales, zeros, K, N, Y, ws, s);
-        case 3: return launch_t<XT, 3>(w, map, X, M, scales, zeros, K, N, Y, ws, s);
-        default: return launch_t<XT, 4>(w, map, X, M, scales, zeros, K, N, Y, ws, s);
+        case 1: return launch_t<XT, 1, 16>(w, map, X, M, scales, zeros, K, N, Y, ws, s);
+        case 2: return launch_t<XT, 2, 16>(w, map, X, M, scales, zeros, K, N, Y, ws, s);
+        case 3: return launch_t<XT, 3, 8>(w, map, X, M, scales, zeros, K, N, Y, ws, s);
+        default: return launch_t<XT, 4, 8>(w, map, X, M, scales, zeros, K, N, Y, ws, s);
     }
 }
 
