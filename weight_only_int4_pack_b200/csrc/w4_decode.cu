@@ -343,11 +343,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     int cur_rb = -1, first_ks = 0, last_ks = -1;
     uint32_t xph = 0;  // flushes done (pair exchange parity)
     bool ok = true;
+    int pending[2];    // row blocks whose partials this warp stored (at most 2 per CTA)
+    int npending = 0;
 
     // Finishes row block rb for this tile's 16 rows.  Waits are bounded; no
     // step waits on a warp of another tile.  A row block split between CTAs
     // has one arrival counter per (row block, tile), and the last warp to
-    // arrive adds the partials in CTA order.
+    // arrive adds the partials in CTA order (finish_partials).
     auto flush = [&](int rb) -> bool {
         if (H == 2) {
             float *xc = xchg + (tile * 32 + lane) * 4 * MT;
@@ -387,7 +389,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                 }
             return true;
         }
-        // partial: slot 0 for the CTA's first row block, 1 for its last
+        // partial: slot 0 for the CTA's first row block, 1 for its last.  Only
+        // the store happens here; the arrival and the final sum wait until the
+        // CTA's units are all done (finish_partials), so the warp goes on.
         const int slot = 2 * c + (rb == u0 / wk.KS ? 0 : 1);
         float *dst = partial + (int64_t)slot * kUnitRows * M;
 #pragma unroll
@@ -398,29 +402,40 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                 const int m = 8 * mt + 2 * t + (i & 1);
                 if (m < M) dst[r * M + m] = acc[mt][i];
             }
-        __threadfence();
-        __syncwarp();
-        const int cf = owner(wk, rb * wk.KS), cl = owner(wk, (rb + 1) * wk.KS - 1);
-        unsigned *cnt = counters + rb * 8 + tile;
-        unsigned prev = 0;
-        if (lane == 0) prev = atomicAdd(cnt, 1u);
-        prev = __shfl_sync(0xffffffffu, prev, 0);
-        if (prev != (unsigned)(cl - cf)) return true;
-        __threadfence();
-        for (int e = lane; e < 16 * M; e += 32) {
-            const int r = 16 * tile + (e & 15), m = e >> 4;
-            const int n = n0 + r;
-            if (n >= N) continue;
-            float v = 0.0f;
-            for (int cc = cf; cc <= cl; ++cc) {
-                const int sl = 2 * cc + (rb == range_start(wk, cc) / wk.KS ? 0 : 1);
-                v += __ldcg(partial + ((int64_t)sl * kUnitRows + r) * M + m);
-            }
-            store_out<XT>(Y, (int64_t)m * N + n, v);
-        }
-        __syncwarp();
-        if (lane == 0) *cnt = 0u;  // re-arm for the next call
+        pending[npending++] = rb;
         return true;
+    };
+
+    // Arrives on the counters of the row blocks whose partials this warp
+    // stored; the last warp to arrive on one adds its partials in CTA order.
+    auto finish_partials = [&]() {
+        if (npending == 0) return;
+        __threadfence();
+        __syncwarp();
+        for (int q = 0; q < npending; ++q) {
+            const int rb = pending[q];
+            const int n0 = rb * kUnitRows;
+            const int cf = owner(wk, rb * wk.KS), cl = owner(wk, (rb + 1) * wk.KS - 1);
+            unsigned *cnt = counters + rb * 8 + tile;
+            unsigned prev = 0;
+            if (lane == 0) prev = atomicAdd(cnt, 1u);
+            prev = __shfl_sync(0xffffffffu, prev, 0);
+            if (prev != (unsigned)(cl - cf)) continue;
+            __threadfence();
+            for (int e = lane; e < 16 * M; e += 32) {
+                const int r = 16 * tile + (e & 15), m = e >> 4;
+                const int n = n0 + r;
+                if (n >= N) continue;
+                float v = 0.0f;
+                for (int cc = cf; cc <= cl; ++cc) {
+                    const int sl = 2 * cc + (rb == range_start(wk, cc) / wk.KS ? 0 : 1);
+                    v += __ldcg(partial + ((int64_t)sl * kUnitRows + r) * M + m);
+                }
+                store_out<XT>(Y, (int64_t)m * N + n, v);
+            }
+            __syncwarp();
+            if (lane == 0) *cnt = 0u;  // re-arm for the next call
+        }
     };
 
     // scales and zero points of one unit for this thread's two rows and
@@ -512,8 +527,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                 uint4 xv[MT];
                 const int ch = ((xsw + j) ^ g) << 4;
 #pragma unroll
-                for (int mt = 0; mt < MT; ++mt)
-                    xv[mt] = *reinterpret_cast<const uint4 *>(xg + mt * 1024 + ch);
+                for (int mt = 0; mt < MT; ++mt) {
+                    // rows >= M are zero: those lanes skip the shared-memory read
+                    xv[mt] = make_uint4(0, 0, 0, 0);
+                    if (8 * mt + g < M) xv[mt] = *reinterpret_cast<const uint4 *>(xg + mt * 1024 + ch);
+                }
                 uint32_t pa[4], pb[4];
                 dequant_word<XT>(wav[j], zba[q], zqa[q], pa);
                 dequant_word<XT>(wbv[j], zbb[q], zqb[q], pb);
@@ -542,7 +560,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         rb = nrb;
         ks = nks;
     }
-    if (ok && cur_rb >= 0) flush(cur_rb);
+    if (ok && cur_rb >= 0) ok = flush(cur_rb);
+    if (ok && (H == 1 || half == 0)) finish_partials();
 }
 
 // ---- host side --------------------------------------------------------------------------
