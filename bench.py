@@ -88,6 +88,14 @@ def sum_over_ranks(x: float) -> float:
     return x
 
 
+def aggregate_rate(bytes_local: float, ms_local: float) -> float:
+    """Whole-job throughput in TB/s: the bytes all ranks processed divided by
+    the slowest rank's time (every rank calls this, in the same order)."""
+    ms = max_over_ranks(ms_local)
+    total = sum_over_ranks(bytes_local)
+    return total / (ms * 1e-3) / 1e12
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples while the timed region runs."""
 
@@ -292,10 +300,9 @@ def run_ours(args, ws_, rank, local):
         for i in range(n % block):
             graphs[i % copies].replay()
 
-    ms, clocks = timed_block(run_steps, args.steps, args.warmup, sampler=ClockSampler(local))
-    ms = max_over_ranks(ms)
-    total_bytes = sum_over_ranks(step_bytes * args.steps)
-    value_tbs = total_bytes / (ms * 1e-3) / 1e12
+    ms_local, clocks = timed_block(run_steps, args.steps, args.warmup, sampler=ClockSampler(local))
+    value_tbs = aggregate_rate(step_bytes * args.steps, ms_local)
+    ms = max_over_ranks(ms_local)
 
     per_layer = []
     for li, N in enumerate(Ns):
@@ -321,9 +328,10 @@ def run_ours(args, ws_, rank, local):
             yh.copy_(Y, non_blocking=True)
 
     e2e_steps = min(args.steps, 2000)
-    e2e_ms, _ = timed(step_e2e, e2e_steps, args.warmup)
-    e2e_ms = max_over_ranks(e2e_ms)
-    e2e = {"value": round(sum_over_ranks(step_bytes * e2e_steps) / (e2e_ms * 1e-3) / 1e12, 4),
+    e2e_ms_local, _ = timed(step_e2e, e2e_steps, args.warmup)
+    e2e_value = aggregate_rate(step_bytes * e2e_steps, e2e_ms_local)
+    e2e_ms = max_over_ranks(e2e_ms_local)
+    e2e = {"value": round(e2e_value, 4),
            "unit": "TB/s", "h2d_bytes_per_step": int(X.numel() * 2),
            "d2h_bytes_per_step": int(sum(N * 2 for N in Ns)),
            "ms_per_step": round(e2e_ms / e2e_steps, 5)}

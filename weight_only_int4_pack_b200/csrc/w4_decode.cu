@@ -56,13 +56,9 @@ constexpr int kGroup = 128;
 constexpr int kUnitRows = 128;                      // weight rows per unit (= TMEM lanes)
 constexpr int kUnitK = 256;                         // k per unit: two groups, 128 bytes per row
 constexpr int kUnitBytes = kUnitRows * kUnitK / 2;  // 16 KB of codes
-constexpr int kSZBytes = kUnitRows * 2 * 4;         // scales (or zeros) of a unit: [128][2] fp32
-constexpr int kThreads = 320;                       // producer, MMA, two dequant warpgroups
+constexpr int kSZBytes = kUnitRows * 2 * 4;         // zero points (or scales) of a unit: [128][2] fp32
 constexpr int kTmemCols = 512;
-// TMEM columns: A operand [group][buffer] 64 columns each (128 k of 16-bit
-// pairs), then the fp32 partials [group][buffer] of N columns each.
-constexpr int kAColsPerGroup = 64;
-constexpr int kDBase = 256;
+constexpr int kAColsPerGroup = 64;  // A operand of one group: 128 k of 16-bit pairs
 // Workspace: arrival counters (one per row block and 32-row warp) first,
 // then two partial slots per CTA ([2 * ctas][128 rows][M] fp32).  The counter
 // area is fixed so that one workspace serves calls of any shape; row-block
@@ -109,14 +105,37 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Up to 64 polls of the barrier in a tight loop (five instructions a poll):
+// true as soon as the phase with `parity` has completed.
+__device__ __forceinline__ bool mbar_poll64(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t.reg .u32 n;\n\t"
+        "mov.u32 n, 64;\n"
+        "W4_POLL_%=:\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "@p bra W4_DONE_%=;\n\t"
+        "sub.u32 n, n, 1;\n\t"
+        "setp.ne.u32 q, n, 0;\n\t"
+        "@q bra W4_POLL_%=;\n"
+        "W4_DONE_%=:\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait: true once the phase with `parity` has completed; false if the
 // CTA aborted or the wait ran out (then the abort flag and status are set).
+// The abort flag and the clock are looked at every 64 polls only, so that
+// waiting warps take few issue slots from the working ones.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
                                           unsigned *status) {
     if (mbar_try(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     while (true) {
-        if (mbar_try(bar, parity)) return true;
+        if (mbar_poll64(bar, parity)) return true;
         if (*abort_flag) return false;
         if (globaltimer() - t0 > kWaitNs) {
             *abort_flag = 1;
@@ -148,6 +167,17 @@ __device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
 // The mbarrier gets one arrival once all of this thread's cp.async copies landed.
 __device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// true in exactly one lane of the (fully active) warp
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
 }
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -193,13 +223,6 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
                  : "memory");
 }
 
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t *r) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
-                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
-                 "r"(r[7])
-                 : "memory");
-}
-
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
@@ -228,30 +251,83 @@ __device__ __forceinline__ void zero_bias(float z, uint32_t &zb, uint32_t &zq) {
     }
 }
 
-// One packed word (k = 8j..8j+7 of a row) -> four registers holding the exact
-// pairs (u - z) of k = {0,1}, {2,3}, {4,5}, {6,7} (low half = even k).  The
-// packed layout keeps k = 8j+{2i, 2i+1} in nibbles i and i+4 of the word.
+// Dequantizes 8 packed words (64 codes of one row, k = 8i .. 8i + 7 in word
+// i) and stores the 32 exact pairs (u - z) to TMEM columns taddr ..
+// taddr + 31 of this thread's lane, in one block: the 32 results are produced
+// straight into the store's registers.  mask_lo, mask_hi and magic come in
+// registers so that each nibble pair costs one LOP3.  fp16: pairs {0,1} and
+// {4,5} come from the low nibbles of the word and of the word >> 8, minus
+// (1024 + z); pairs {2,3} and {6,7} from the high nibbles, times 1/16 minus
+// (64 + z).  bf16: nibble i of each half (word >> 4i), minus (128 + z).
 template <int XT>
-__device__ __forceinline__ void dequant_word(uint32_t w, uint32_t zb, uint32_t zq, uint32_t *p) {
+__device__ __forceinline__ void dequant8_store(uint32_t taddr, const uint32_t (&w)[8], uint32_t zb,
+                                               uint32_t zq) {
+    uint32_t mlo, mhi, magic, sixteenth;
+    asm("mov.b32 %0, 0x000F000F;" : "=r"(mlo));
+    asm("mov.b32 %0, 0x00F000F0;" : "=r"(mhi));
     if (XT == W4_F16) {
-        const uint32_t magic = 0x64006400u;      // {1024, 1024}
-        const uint32_t sixteenth = 0x2C002C00u;  // {1/16, 1/16}
-        const uint32_t lo0 = (w & 0x000F000Fu) | magic;
-        const uint32_t hi0 = (w & 0x00F000F0u) | magic;
-        const uint32_t w8 = w >> 8;
-        const uint32_t lo1 = (w8 & 0x000F000Fu) | magic;
-        const uint32_t hi1 = (w8 & 0x00F000F0u) | magic;
-        asm("sub.f16x2 %0, %1, %2;" : "=r"(p[0]) : "r"(lo0), "r"(zb));
-        asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(p[1]) : "r"(hi0), "r"(sixteenth), "r"(zq));
-        asm("sub.f16x2 %0, %1, %2;" : "=r"(p[2]) : "r"(lo1), "r"(zb));
-        asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(p[3]) : "r"(hi1), "r"(sixteenth), "r"(zq));
+        asm("mov.b32 %0, 0x64006400;" : "=r"(magic));
+        asm("mov.b32 %0, 0x2C002C00;" : "=r"(sixteenth));
+#define W4_F16_WORD(i)                                                   \
+    "lop3.b32 t" #i "a, %" #i ", mlo, magic, 0xEA;\n\t"                  \
+    "lop3.b32 t" #i "b, %" #i ", mhi, magic, 0xEA;\n\t"                  \
+    "shr.b32 x, %" #i ", 8;\n\t"                                         \
+    "lop3.b32 t" #i "c, x, mlo, magic, 0xEA;\n\t"                        \
+    "lop3.b32 t" #i "d, x, mhi, magic, 0xEA;\n\t"                        \
+    "sub.f16x2 t" #i "a, t" #i "a, zb;\n\t"                               \
+    "fma.rn.f16x2 t" #i "b, t" #i "b, six, zq;\n\t"                       \
+    "sub.f16x2 t" #i "c, t" #i "c, zb;\n\t"                               \
+    "fma.rn.f16x2 t" #i "d, t" #i "d, six, zq;\n\t"
+        asm volatile(
+            "{\n\t"
+            ".reg .b32 t0a, t0b, t0c, t0d, t1a, t1b, t1c, t1d, t2a, t2b, t2c, t2d, t3a, t3b, t3c, t3d;\n\t"
+            ".reg .b32 t4a, t4b, t4c, t4d, t5a, t5b, t5c, t5d, t6a, t6b, t6c, t6d, t7a, t7b, t7c, t7d;\n\t"
+            ".reg .b32 x, mlo, mhi, magic, six, zb, zq;\n\t"
+            "mov.b32 mlo, %9;\n\tmov.b32 mhi, %10;\n\tmov.b32 magic, %11;\n\t"
+            "mov.b32 six, %12;\n\tmov.b32 zb, %13;\n\tmov.b32 zq, %14;\n\t"
+            W4_F16_WORD(0) W4_F16_WORD(1) W4_F16_WORD(2) W4_F16_WORD(3)
+            W4_F16_WORD(4) W4_F16_WORD(5) W4_F16_WORD(6) W4_F16_WORD(7)
+            "tcgen05.st.sync.aligned.32x32b.x32.b32 [%8], {t0a, t0b, t0c, t0d, t1a, t1b, t1c, t1d, "
+            "t2a, t2b, t2c, t2d, t3a, t3b, t3c, t3d, t4a, t4b, t4c, t4d, t5a, t5b, t5c, t5d, "
+            "t6a, t6b, t6c, t6d, t7a, t7b, t7c, t7d};\n\t"
+            "}" ::"r"(w[0]),
+            "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]), "r"(taddr),
+            "r"(mlo), "r"(mhi), "r"(magic), "r"(sixteenth), "r"(zb), "r"(zq)
+            : "memory");
+#undef W4_F16_WORD
     } else {
-        const uint32_t magic = 0x43004300u;  // {128, 128} in bf16
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t v = ((w >> (4 * i)) & 0x000F000Fu) | magic;
-            asm("sub.bf16x2 %0, %1, %2;" : "=r"(p[i]) : "r"(v), "r"(zb));
-        }
+        asm("mov.b32 %0, 0x43004300;" : "=r"(magic));
+#define W4_BF16_WORD(i)                                                  \
+    "lop3.b32 t" #i "a, %" #i ", mlo, magic, 0xEA;\n\t"                  \
+    "shr.b32 x, %" #i ", 4;\n\t"                                         \
+    "lop3.b32 t" #i "b, x, mlo, magic, 0xEA;\n\t"                        \
+    "shr.b32 x, %" #i ", 8;\n\t"                                         \
+    "lop3.b32 t" #i "c, x, mlo, magic, 0xEA;\n\t"                        \
+    "shr.b32 x, %" #i ", 12;\n\t"                                        \
+    "lop3.b32 t" #i "d, x, mlo, magic, 0xEA;\n\t"                        \
+    "sub.bf16x2 t" #i "a, t" #i "a, zb;\n\t"                              \
+    "sub.bf16x2 t" #i "b, t" #i "b, zb;\n\t"                              \
+    "sub.bf16x2 t" #i "c, t" #i "c, zb;\n\t"                              \
+    "sub.bf16x2 t" #i "d, t" #i "d, zb;\n\t"
+        asm volatile(
+            "{\n\t"
+            ".reg .b32 t0a, t0b, t0c, t0d, t1a, t1b, t1c, t1d, t2a, t2b, t2c, t2d, t3a, t3b, t3c, t3d;\n\t"
+            ".reg .b32 t4a, t4b, t4c, t4d, t5a, t5b, t5c, t5d, t6a, t6b, t6c, t6d, t7a, t7b, t7c, t7d;\n\t"
+            ".reg .b32 x, mlo, magic, zb;\n\t"
+            "mov.b32 mlo, %9;\n\tmov.b32 magic, %10;\n\tmov.b32 zb, %11;\n\t"
+            W4_BF16_WORD(0) W4_BF16_WORD(1) W4_BF16_WORD(2) W4_BF16_WORD(3)
+            W4_BF16_WORD(4) W4_BF16_WORD(5) W4_BF16_WORD(6) W4_BF16_WORD(7)
+            "tcgen05.st.sync.aligned.32x32b.x32.b32 [%8], {t0a, t0b, t0c, t0d, t1a, t1b, t1c, t1d, "
+            "t2a, t2b, t2c, t2d, t3a, t3b, t3c, t3d, t4a, t4b, t4c, t4d, t5a, t5b, t5c, t5d, "
+            "t6a, t6b, t6c, t6d, t7a, t7b, t7c, t7d};\n\t"
+            "}" ::"r"(w[0]),
+            "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]), "r"(taddr),
+            "r"(mlo), "r"(magic), "r"(zb)
+            : "memory");
+#undef W4_BF16_WORD
+        (void)zq;
+        (void)mhi;
+        (void)sixteenth;
     }
 }
 
@@ -288,43 +364,61 @@ __device__ __forceinline__ int owner(const Work &w, int u) {
 
 // NN: MMA N (16 or 32) = X rows staged per unit (rows >= M are zero).
 // Stage: codes [128][128 B] (swizzled) | X: four 64-k boxes [NN][128 B]
-// (swizzled) | scales [128][2] | zeros [128][2].
+// (swizzled) | zero points [128][2] fp32.
+//
+// Slots: unit `it` of a CTA's range uses TMEM slot it % kSlots, which holds
+// its A operand (both groups, 2 x 64 columns) and its two fp32 partials
+// (2 x NN columns).  A slot is reused by unit it + kSlots once the MMAs of
+// unit it are done and its partials have been read.
 template <int NN>
 struct Cfg {
     static constexpr int kXBox = NN * 128;
-    static constexpr int kSZ = kUnitBytes + 4 * kXBox;
-    static constexpr int kBytes = kSZ + 2 * kSZBytes;
+    static constexpr int kZOff = kUnitBytes + 4 * kXBox;
+    static constexpr int kBytes = kZOff + kSZBytes;
     static constexpr int kTmaBytes = kUnitBytes + 4 * kXBox;
-    static constexpr int kStages = (176 * 1024) / kBytes < 8 ? (176 * 1024) / kBytes : 8;
-    static constexpr int kXchg = kUnitRows * NN * 4;  // second warpgroup's half at a flush
-    static constexpr int kSmem = kStages * kBytes + 1024 + 512 + kXchg;
+    static constexpr int kXchgBytes = 4 * NN * 32 * 4;  // [quarter][m][lane] fp32
+    static constexpr int kStages =
+        (200 * 1024 - kXchgBytes) / kBytes < 8 ? (200 * 1024 - kXchgBytes) / kBytes : 8;
+    static constexpr int kSmem = kStages * kBytes + 1024 + 512 + kXchgBytes;
+    static constexpr int kSlots = kTmemCols / (2 * kAColsPerGroup + 2 * NN);
+    static constexpr int kDBase = kSlots * 2 * kAColsPerGroup;
+    static_assert(kSlots >= 2 && kSlots <= 3, "TMEM slots");
+    static_assert(kDBase + kSlots * 2 * NN <= kTmemCols, "TMEM columns");
 };
 
 struct Shared {
-    uint64_t full[8];      // codes + X (TMA bytes) and scales/zeros (cp.async) landed
-    uint64_t empty[8];     // both groups' MMAs of the stage done
-    uint64_t afull[2][2];  // [group][buffer] A operand stored in TMEM (128 threads)
-    uint64_t afree[2][2];  // its MMAs done (commit)
-    uint64_t dfull[2][2];  // [group][buffer] partial complete (commit)
-    uint64_t dfree[2][2];  // partial read (128 threads)
-    uint64_t xfull, xfree; // warpgroup 1 -> 0 exchange at a flush (128 threads each)
+    uint64_t full[8];   // stage: codes + X (TMA bytes) and zero points (cp.async) landed
+    uint64_t empty[8];  // stage: the unit's MMAs done (commit)
+    uint64_t ready[3];  // slot: A stored and the previous partials read (4 dequant warps)
+    uint64_t mdone[3];  // slot: the unit's MMAs done (commit): A free, partials complete
+    uint64_t xfull[4];  // lane quarter: group-1 accumulators of a row block in xbuf
+    uint64_t xfree[4];  // lane quarter: xbuf read
     uint32_t tmem_base;
     int abort_flag;
 };
 
+// Warp roles (10 warps): 0 producer, 1 TMEM allocator + MMA issuer,
+// 2..9 dequant (warp w: TMEM lane quarter w % 4, the units of parity
+// (w - 2) / 4), which also fold the partials of their rows.
+constexpr int kDequantWarps = 8;
+constexpr int kThreads = 32 * (2 + kDequantWarps);
+
+// Launch bounds of 384 threads cap the registers at 168 a thread: up to three
+// of the 10 warps share one SM sub-partition (16K registers).
 template <int XT, int NN>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(384, 1)
 decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
               int M, const float *__restrict__ scales, const float *__restrict__ zeros, int K, int N,
               void *__restrict__ Y, unsigned *__restrict__ counters, float *__restrict__ partial,
               const Work wk, unsigned *__restrict__ status) {
     using C = Cfg<NN>;
     constexpr int S = C::kStages;
+    constexpr int R = C::kSlots;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
     Shared *sh = reinterpret_cast<Shared *>(ring + S * C::kBytes);
-    float *xchg = reinterpret_cast<float *>(ring + S * C::kBytes + 512);
+    float *xbuf = reinterpret_cast<float *>(ring + S * C::kBytes + 512);
     volatile int *abort_flag = &sh->abort_flag;
 
     const int warp = threadIdx.x >> 5;
@@ -332,6 +426,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     const int c = blockIdx.x;
     const int u0 = range_start(wk, c);
     const int u1 = range_start(wk, c + 1);
+    const int nu = u1 - u0;
     const int G = wk.G;
 
     if (threadIdx.x == 0) {
@@ -339,15 +434,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             mbar_init(smem_u32(&sh->full[s]), 1 + 32);  // TMA arrive_tx + 32 cp.async arrivals
             mbar_init(smem_u32(&sh->empty[s]), 1);
         }
-        for (int h = 0; h < 2; ++h)
-            for (int b = 0; b < 2; ++b) {
-                mbar_init(smem_u32(&sh->afull[h][b]), 128);
-                mbar_init(smem_u32(&sh->afree[h][b]), 1);
-                mbar_init(smem_u32(&sh->dfull[h][b]), 1);
-                mbar_init(smem_u32(&sh->dfree[h][b]), 128);
-            }
-        mbar_init(smem_u32(&sh->xfull), 128);
-        mbar_init(smem_u32(&sh->xfree), 128);
+        for (int j = 0; j < R; ++j) {
+            mbar_init(smem_u32(&sh->ready[j]), 4);  // the unit's four dequant warps
+            mbar_init(smem_u32(&sh->mdone[j]), 1);
+        }
+        for (int q = 0; q < 4; ++q) {
+            mbar_init(smem_u32(&sh->xfull[q]), 1);
+            mbar_init(smem_u32(&sh->xfree[q]), 1);
+        }
         sh->abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -366,44 +460,49 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
 
     if (warp == 0) {
         // ---------------- producer ----------------
-        // Codes and X by TMA (lane 0), the unit's scales and zero points by
-        // cp.async (four rows per lane); every lane arrives on the stage's full
-        // barrier once its copies have landed.
-        auto issue_sz = [&](int u, uint8_t *st, uint32_t fb) {
-            const int rb = u / wk.KS, ks = u % wk.KS;
-            const int g0 = 2 * ks, g1 = min(2 * ks + 1, G - 1);
-            float *ss = reinterpret_cast<float *>(st + C::kSZ);
-            float *zz = ss + 2 * kUnitRows;
+        // Codes and X by TMA (lane 0); the unit's zero points by cp.async (four
+        // rows per lane); every lane arrives on the stage's full barrier once
+        // its copies have landed.
+        auto issue_sz = [&](int rb, int ks, uint8_t *st, uint32_t fb) {
+            if (zeros) {
+                const int g0 = 2 * ks, g1 = min(2 * ks + 1, G - 1);
+                float *zz = reinterpret_cast<float *>(st + C::kZOff);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int r = lane + 32 * q;
-                const int64_t n = min(rb * kUnitRows + r, N - 1);
-                cp_async4(smem_u32(ss + 2 * r), scales + n * G + g0);
-                cp_async4(smem_u32(ss + 2 * r + 1), scales + n * G + g1);
-                if (zeros) {
+                for (int q = 0; q < 4; ++q) {
+                    const int r = lane + 32 * q;
+                    const int64_t n = min(rb * kUnitRows + r, N - 1);
                     cp_async4(smem_u32(zz + 2 * r), zeros + n * G + g0);
                     cp_async4(smem_u32(zz + 2 * r + 1), zeros + n * G + g1);
                 }
             }
             cp_async_arrive(fb);
         };
-        auto issue_x = [&](int u, uint8_t *st, uint32_t fb) {
-            const int ks = u % wk.KS;
+        auto issue_x = [&](int ks, uint8_t *st, uint32_t fb) {
 #pragma unroll
             for (int b = 0; b < 4; ++b)
                 tma_load_2d(smem_u32(st + kUnitBytes + b * C::kXBox), &tmap_x, ks * kUnitK + 64 * b, 0,
                             fb);
         };
-        // The packed weights are inputs no earlier kernel writes: the first ring
-        // of codes is requested before waiting for the preceding kernel.
-        const int pre = min(S, u1 - u0);
+        auto issue_w = [&](int rb, int ks, uint8_t *st, uint32_t fb) {
+            mbar_arrive_tx(fb, C::kTmaBytes);
+            tma_load_2d(smem_u32(st), &tmap_w, ks * (kUnitK / 2), rb * kUnitRows, fb);
+        };
+        // (rb, ks): row block and k step of the next unit to issue
+        int rb = u0 / wk.KS, ks = u0 - (u0 / wk.KS) * wk.KS;
+        // The packed weights are inputs no earlier kernel writes: the codes of
+        // the first two units are requested before waiting for the preceding
+        // kernel; the X slices, zero points and scales of the first units go
+        // out before the rest of the first ring, so that unit 0 lands early.
+        const int pre = min(S, nu);
+        const int early = min(2, pre);
         if (lane == 0) {
-            for (int it = 0; it < pre; ++it) {
-                const int u = u0 + it;
-                const uint32_t fb = smem_u32(&sh->full[it]);
-                mbar_arrive_tx(fb, C::kTmaBytes);
-                tma_load_2d(smem_u32(ring + it * C::kBytes), &tmap_w, (u % wk.KS) * (kUnitK / 2),
-                            (u / wk.KS) * kUnitRows, fb);
+            int rb2 = rb, ks2 = ks;
+            for (int it = 0; it < early; ++it) {
+                issue_w(rb2, ks2, ring + it * C::kBytes, smem_u32(&sh->full[it]));
+                if (++ks2 == wk.KS) {
+                    ks2 = 0;
+                    ++rb2;
+                }
             }
         }
         __syncwarp();
@@ -411,28 +510,40 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         for (int it = 0; it < pre; ++it) {
             uint8_t *st = ring + it * C::kBytes;
             const uint32_t fb = smem_u32(&sh->full[it]);
-            if (lane == 0) issue_x(u0 + it, st, fb);
-            issue_sz(u0 + it, st, fb);
+            if (lane == 0) {
+                if (it >= early) issue_w(rb, ks, st, fb);
+                issue_x(ks, st, fb);
+            }
+            issue_sz(rb, ks, st, fb);
+            if (++ks == wk.KS) {
+                ks = 0;
+                ++rb;
+            }
         }
-        int u = u0 + pre;
-        for (; u < u1; ++u) {
-            const int it = u - u0;
-            const int s = it % S;
-            const uint32_t ph = (it / S) & 1;
+        int it = pre;
+        int s = 0;        // stage of unit it (it >= pre only runs when pre == S)
+        uint32_t ph = 1;  // its fill parity
+        for (; it < nu; ++it) {
             if (!warp_wait(smem_u32(&sh->empty[s]), ph ^ 1, abort_flag, status)) break;
             uint8_t *st = ring + s * C::kBytes;
             const uint32_t fb = smem_u32(&sh->full[s]);
             if (lane == 0) {
-                mbar_arrive_tx(fb, C::kTmaBytes);
-                tma_load_2d(smem_u32(st), &tmap_w, (u % wk.KS) * (kUnitK / 2), (u / wk.KS) * kUnitRows,
-                            fb);
-                issue_x(u, st, fb);
+                issue_w(rb, ks, st, fb);
+                issue_x(ks, st, fb);
             }
-            issue_sz(u, st, fb);
+            issue_sz(rb, ks, st, fb);
+            if (++ks == wk.KS) {
+                ks = 0;
+                ++rb;
+            }
+            if (++s == S) {
+                s = 0;
+                ph ^= 1;
+            }
         }
         // wait (bounded) for the copies still in flight before the CTA may exit
         if (lane == 0) {
-            for (int j = (u - u0 > S ? u - u0 - S : 0); j < u - u0; ++j) {
+            for (int j = (it > S ? it - S : 0); j < it; ++j) {
                 const unsigned long long t0 = globaltimer();
                 while (!mbar_try(smem_u32(&sh->full[j % S]), (j / S) & 1) &&
                        globaltimer() - t0 < kWaitNs) {
@@ -442,107 +553,114 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         __syncwarp();
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
-        if (lane == 0) {
-            constexpr uint32_t idesc = instr_desc<XT, NN>();
-            uint32_t n_mma[2] = {0, 0};  // group MMAs issued, per warpgroup
-            bool ok = true;
-            int u = u0;
-            for (; u < u1 && ok; ++u) {
-                const int it = u - u0;
-                const int s = it % S;
-                const uint32_t ph = (it / S) & 1;
-                const int ks = u % wk.KS;
-                if (!mbar_wait(smem_u32(&sh->full[s]), ph, abort_flag, status)) break;
-                const uint32_t xs = smem_u32(ring + s * C::kBytes + kUnitBytes);
-                for (int h = 0; h < 2; ++h) {
-                    if (2 * ks + h >= G) break;  // a last unit with one group
-                    const uint32_t b = n_mma[h] & 1, pb = (n_mma[h] >> 1) & 1;
-                    if (!mbar_wait(smem_u32(&sh->afull[h][b]), pb, abort_flag, status) ||
-                        !mbar_wait(smem_u32(&sh->dfree[h][b]), pb ^ 1, abort_flag, status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t ta = tmem + (uint32_t)((2 * h + b) * kAColsPerGroup);
-                    const uint32_t td = tmem + (uint32_t)(kDBase + (2 * h + b) * NN);
+        // The whole warp takes the waits (warp-uniform operands stay in
+        // uniform registers); one elected lane issues.  The tensor pipe queues
+        // only a few MMAs, so the wait for unit it + 1 is taken while the last
+        // four MMAs of unit it are still to be issued: the pipe never runs dry
+        // between units when the next unit is ready.  Each unit waits on one
+        // barrier: its slot's `ready` (A stored, previous partials read).  Its
+        // X comes from the stage the dequant warps waited for before they
+        // arrived.
+        constexpr uint32_t idesc = instr_desc<XT, NN>();
+        const bool leader = elect_one();
+        const uint64_t xdesc0 = sw128_desc(smem_u32(ring + kUnitBytes));
+        int done = -1;  // last unit whose MMAs are tracked by its empty barrier
+        bool ok = nu > 0 && warp_wait(smem_u32(&sh->ready[0]), 0, abort_flag, status);
+        int ks = u0 - (u0 / wk.KS) * wk.KS;  // k step of unit it
+        int s = 0, j = 0;                    // its stage and slot
+        int jn = 1;                          // slot of unit it + 1 and its ready parity
+        uint32_t pn = 0;
+        for (int it = 0; it < nu && ok; ++it) {
+            const bool two = 2 * ks + 1 < G;  // false: a last unit with one group
+            tc_fence_after();
+            // stage s's X boxes: descriptor start address advances in 16-byte units
+            const uint64_t xd = xdesc0 + (uint64_t)((s * C::kBytes) >> 4);
+            const uint32_t ta0 = tmem + (uint32_t)(2 * j * kAColsPerGroup);
+            const uint32_t ta1 = ta0 + kAColsPerGroup;
+            const uint32_t td0 = tmem + (uint32_t)(C::kDBase + 2 * j * NN);
+            const uint32_t td1 = td0 + NN;
+            // group h, k16 step kb: X box 2h + kb/4, 32 bytes per step in its swizzle row
+            auto issue = [&](int kb) {
+                const uint32_t off0 = (uint32_t)(((kb / 4) * C::kXBox + (kb % 4) * 32) >> 4);
+                const uint32_t off1 = (uint32_t)(((2 + kb / 4) * C::kXBox + (kb % 4) * 32) >> 4);
+                mma_ts(td0, ta0 + 8 * kb, xd + off0, idesc, kb > 0 ? 1u : 0u);
+                if (two) mma_ts(td1, ta1 + 8 * kb, xd + off1, idesc, kb > 0 ? 1u : 0u);
+            };
+            if (leader) {
 #pragma unroll
-                    for (int kb = 0; kb < 8; ++kb) {
-                        // X box 2h + kb/4, 16 k (32 bytes) per step inside the swizzle row
-                        const uint32_t xa = xs + (2 * h + kb / 4) * C::kXBox + (kb % 4) * 32;
-                        mma_ts(td, ta + 8 * kb, sw128_desc(xa), idesc, kb > 0 ? 1u : 0u);
-                    }
-                    mma_commit(smem_u32(&sh->afree[h][b]));
-                    mma_commit(smem_u32(&sh->dfull[h][b]));
-                    ++n_mma[h];
-                }
-                if (ok) mma_commit(smem_u32(&sh->empty[s]));
+                for (int kb = 0; kb < 6; ++kb) issue(kb);
             }
-            // drain: wait (bounded) until the last issued MMAs have completed
-            if (u > u0) {
-                const int j = u - 1 - u0;
-                const unsigned long long t0 = globaltimer();
-                while (!mbar_try(smem_u32(&sh->empty[j % S]), (j / S) & 1) &&
-                       globaltimer() - t0 < kWaitNs) {
-                }
+            __syncwarp();
+            bool ok_next = true;
+            if (it + 1 < nu) ok_next = warp_wait(smem_u32(&sh->ready[jn]), pn, abort_flag, status);
+            if (leader) {
+                issue(6);
+                issue(7);
+                mma_commit(smem_u32(&sh->mdone[j]));
+                mma_commit(smem_u32(&sh->empty[s]));
+            }
+            __syncwarp();
+            done = it;
+            ok = ok_next;
+            if (++ks == wk.KS) ks = 0;
+            if (++s == S) s = 0;
+            j = jn;
+            if (++jn == R) {
+                jn = 0;
+                pn ^= 1;
+            }
+        }
+        // drain: wait (bounded) until the last issued MMAs have completed
+        if (done >= 0 && lane == 0) {
+            const unsigned long long t0 = globaltimer();
+            while (!mbar_try(smem_u32(&sh->empty[done % S]), (done / S) & 1) &&
+                   globaltimer() - t0 < kWaitNs) {
             }
         }
         __syncwarp();
     } else {
-        // ---------------- dequant + accumulate: two warpgroups ----------------
-        const int h = (warp - 2) >> 2;               // group of each unit this warpgroup owns
-        const int q = warp & 3;                      // TMEM lane quarter of this warp
-        const int r = 32 * q + lane;                 // weight row of the unit (= TMEM lane)
+        // ---------------- dequant + fold: 8 warps ----------------
+        // Warp (q, p) owns rows r = 32q..32q+31 (its TMEM lane quarter) and the
+        // units of parity p of the CTA's range.  For such a unit it, it
+        // dequantizes the row's 256 codes (both groups) into the slot's A
+        // operand, after first adding scale * partial of the slot's previous
+        // unit (it - R, done in the tensor pipe) into its fp32 accumulators.
+        // Both warps of a quarter follow every unit's row block, so that at
+        // each row-block boundary both hand over their sums: the p = 1 warp
+        // through xbuf to the p = 0 warp, which writes Y (or its CTA's
+        // partial of a row block split between CTAs).
+        const int p = (warp - 2) >> 2;
+        const int q = warp & 3;
+        const int r = 32 * q + lane;
         const uint32_t lanebase = (uint32_t)(32 * q) << 16;
         const int swz = r & 7;
         float acc[NN];
-        int cur_rb = -1, first_ks = 0, last_ks = -1;
-        uint32_t n_a = 0, n_d = 0, n_x = 0;          // A stores, partials read, exchanges
-        int pending[2];
-        int npending = 0;
+#pragma unroll
+        for (int i = 0; i < NN; ++i) acc[i] = 0.0f;
+        int cur_rb = -1;      // row block the accumulators belong to
+        int pend0 = -1, pend1 = -1;  // split row blocks stored (p == 0)
+        uint32_t nflush = 0;  // row blocks flushed (xfull / xfree parity)
         bool ok = true;
 
-        // Reads this warpgroup's partial of its previous group and adds it.
-        auto fold = [&](float sc) -> bool {
-            const uint32_t b = n_d & 1, pb = (n_d >> 1) & 1;
-            if (!warp_wait(smem_u32(&sh->dfull[h][b]), pb, abort_flag, status)) return false;
-            tc_fence_after();
-            const uint32_t td = tmem + lanebase + (uint32_t)(kDBase + (2 * h + b) * NN);
-#pragma unroll
-            for (int cc = 0; cc < NN / 16; ++cc) {
-                uint32_t v[16];
-                tmem_ld16(td + 16 * cc, v);
-                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    acc[16 * cc + i] = fmaf(sc, __uint_as_float(v[i]), acc[16 * cc + i]);
-            }
-            tc_fence_before();
-            mbar_arrive(smem_u32(&sh->dfree[h][b]));
-            ++n_d;
-            return true;
-        };
-
-        // Finishes row block rb for this thread's row: the two warpgroups' halves
-        // are added through shared memory, then warpgroup 0 writes Y or stores a
-        // partial (arrival and final sum after the loop, finish_partials).
         auto flush = [&](int rb) -> bool {
-            const uint32_t px = n_x & 1;
-            float *xr = xchg + r * NN;
-            if (h == 1) {
-                if (!warp_wait(smem_u32(&sh->xfree), px ^ 1, abort_flag, status)) return false;
+            float *xb = xbuf + q * NN * 32 + lane;
+            const uint32_t par = nflush & 1;
+            ++nflush;
+            if (p == 1) {
+                if (!warp_wait(smem_u32(&sh->xfree[q]), par ^ 1, abort_flag, status)) return false;
 #pragma unroll
-                for (int i = 0; i < NN; ++i) xr[i] = acc[i];
-                mbar_arrive(smem_u32(&sh->xfull));
-                ++n_x;
+                for (int m = 0; m < NN; ++m) xb[32 * m] = acc[m];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&sh->xfull[q]));
                 return true;
             }
-            if (!warp_wait(smem_u32(&sh->xfull), px, abort_flag, status)) return false;
+            if (!warp_wait(smem_u32(&sh->xfull[q]), par, abort_flag, status)) return false;
 #pragma unroll
-            for (int i = 0; i < NN; ++i) acc[i] += xr[i];
-            mbar_arrive(smem_u32(&sh->xfree));
-            ++n_x;
+            for (int m = 0; m < NN; ++m) acc[m] += xb[32 * m];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sh->xfree[q]));
             const int n = rb * kUnitRows + r;
-            if (first_ks == 0 && last_ks == wk.KS - 1) {
+            if (rb * wk.KS >= u0 && (rb + 1) * wk.KS <= u1) {  // whole row block in this range
                 if (n < N) {
 #pragma unroll
                     for (int m = 0; m < NN; ++m)
@@ -555,31 +673,145 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
 #pragma unroll
             for (int m = 0; m < NN; ++m)
                 if (m < M) dst[m] = acc[m];
-            pending[npending++] = rb;
+            if (pend0 < 0)
+                pend0 = rb;
+            else
+                pend1 = rb;
             return true;
         };
 
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        int ks = u0 - (u0 / wk.KS) * wk.KS;              // unit it: k step
+        int s = 0, j = 0;                                // its stage and slot
+        uint32_t ph = 0, pj = 1;  // full parity; parity of the slot's previous use
+        // unit it - R, the one folded at iteration it (from it = R on): row
+        // block and k step
+        int frb = u0 / wk.KS, fks = u0 - (u0 / wk.KS) * wk.KS;
+        const int last = nu + R;  // iterations nu .. nu + R - 1 only fold
+        for (int it = 0; it < last; ++it) {
+            const bool mine = (it & 1) == p;
+            const bool fold = it >= R;  // unit it - R exists in this range
+            // row-block boundary: unit it - R opens a row block
+            if (fold && frb != cur_rb) {
+                if (cur_rb >= 0 && !flush(cur_rb)) {
+                    ok = false;
+                    break;
+                }
+                cur_rb = frb;
+#pragma unroll
+                for (int i = 0; i < NN; ++i) acc[i] = 0.0f;
+            }
+            if (mine) {
+                const bool unit = it < nu;
+                const bool two = 2 * ks + 1 < G;  // unit it has its second group
+                uint32_t wv[32];
+                uint32_t zb0 = 0, zq0 = 0, zb1 = 0, zq1 = 0;
+                float s0 = 0.0f, s1 = 0.0f;
+                if (fold) {
+                    // scales of the folded unit (row r), from global memory
+                    const int64_t n = min(frb * kUnitRows + r, N - 1);
+                    const float *sp = scales + n * G + 2 * fks;
+                    s0 = __ldg(sp);
+                    s1 = 2 * fks + 1 < G ? __ldg(sp + 1) : 0.0f;
+                }
+                if (unit) {
+                    if (!warp_wait(smem_u32(&sh->full[s]), ph, abort_flag, status)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint8_t *st = ring + s * C::kBytes;
+                    const float *zz = reinterpret_cast<const float *>(st + C::kZOff) + 2 * r;
+                    zero_bias<XT>(zeros ? zz[0] : 8.0f, zb0, zq0);
+                    zero_bias<XT>(zeros ? zz[1] : 8.0f, zb1, zq1);
+                    // the row's 256 codes: eight swizzled 16-byte chunks
+#pragma unroll
+                    for (int cch = 0; cch < 8; ++cch) {
+                        const uint4 v =
+                            *reinterpret_cast<const uint4 *>(st + r * 128 + ((cch ^ swz) << 4));
+                        wv[4 * cch] = v.x;
+                        wv[4 * cch + 1] = v.y;
+                        wv[4 * cch + 2] = v.z;
+                        wv[4 * cch + 3] = v.w;
+                    }
+                }
+                // the slot is free (and its partials complete) once the MMAs of
+                // unit it - R are done
+                if (!warp_wait(smem_u32(&sh->mdone[j]), pj, abort_flag, status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (fold) {
+                    // partial of group 0, then (when the unit has it) of group 1
+                    const uint32_t td = tmem + lanebase + (uint32_t)(C::kDBase + 2 * j * NN);
+                    const int ng = 2 * fks + 1 < G ? 2 : 1;
+                    for (int g = 0; g < ng; ++g) {
+                        const float sg = g == 0 ? s0 : s1;
+#pragma unroll
+                        for (int cc = 0; cc < NN / 16; ++cc) {
+                            uint32_t v[16];
+                            tmem_ld16(td + g * NN + 16 * cc, v);
+                            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+                            for (int i = 0; i < 16; ++i)
+                                acc[16 * cc + i] = fmaf(sg, __uint_as_float(v[i]), acc[16 * cc + i]);
+                        }
+                    }
+                }
+                if (unit) {
+                    const uint32_t ta = tmem + lanebase + (uint32_t)(2 * j * kAColsPerGroup);
+                    dequant8_store<XT>(ta, *reinterpret_cast<const uint32_t(*)[8]>(wv), zb0, zq0);
+                    dequant8_store<XT>(ta + 32, *reinterpret_cast<const uint32_t(*)[8]>(wv + 8), zb0,
+                                       zq0);
+                    if (two) {
+                        dequant8_store<XT>(ta + 64, *reinterpret_cast<const uint32_t(*)[8]>(wv + 16),
+                                           zb1, zq1);
+                        dequant8_store<XT>(ta + 96, *reinterpret_cast<const uint32_t(*)[8]>(wv + 24),
+                                           zb1, zq1);
+                    }
+                    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&sh->ready[j]));
+                }
+            }
+            // advance the cursors of unit it and of unit it - R
+            if (++ks == wk.KS) ks = 0;
+            if (++s == S) {
+                s = 0;
+                ph ^= 1;
+            }
+            if (++j == R) {
+                j = 0;
+                pj ^= 1;
+            }
+            if (fold && ++fks == wk.KS) {
+                fks = 0;
+                ++frb;
+            }
+        }
+        if (ok && cur_rb >= 0) ok = flush(cur_rb);
         // Arrives on the counters of the split row blocks this warp stored; the
         // last warp to arrive on one adds its partials in CTA order.
-        auto finish_partials = [&]() {
-            if (npending == 0) return;
+        if (ok && p == 0 && pend0 >= 0) {
             __threadfence();
             __syncwarp();
-            for (int pi = 0; pi < npending; ++pi) {
-                const int rb = pending[pi];
-                const int cf = owner(wk, rb * wk.KS), cl = owner(wk, (rb + 1) * wk.KS - 1);
-                unsigned *cnt = counters + rb * 8 + q;
+            for (int pi = 0; pi < 2; ++pi) {
+                const int prb = pi == 0 ? pend0 : pend1;
+                if (prb < 0) break;
+                const int cf = owner(wk, prb * wk.KS), cl = owner(wk, (prb + 1) * wk.KS - 1);
+                unsigned *cnt = counters + prb * 8 + q;
                 unsigned prev = 0;
                 if (lane == 0) prev = atomicAdd(cnt, 1u);
                 prev = __shfl_sync(0xffffffffu, prev, 0);
                 if (prev != (unsigned)(cl - cf)) continue;
                 __threadfence();
-                const int n = rb * kUnitRows + r;
+                const int n = prb * kUnitRows + r;
                 if (n < N) {
                     for (int m = 0; m < M; ++m) {
                         float v = 0.0f;
                         for (int cc = cf; cc <= cl; ++cc) {
-                            const int sl = 2 * cc + (rb == range_start(wk, cc) / wk.KS ? 0 : 1);
+                            const int sl = 2 * cc + (prb == range_start(wk, cc) / wk.KS ? 0 : 1);
                             v += __ldcg(partial + ((int64_t)sl * kUnitRows + r) * M + m);
                         }
                         store_out<XT>(Y, (int64_t)m * N + n, v);
@@ -588,88 +820,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                 __syncwarp();
                 if (lane == 0) *cnt = 0u;  // re-arm for the next call
             }
-        };
-
-        asm volatile("griddepcontrol.wait;" ::: "memory");
-        float prev_scale = 0.0f;
-        bool have_prev = false;  // a partial of this warpgroup waits to be folded
-        int rb = u0 / wk.KS;
-        int ks = u0 - rb * wk.KS;
-        for (int u = u0; u < u1; ++u) {
-            const int it = u - u0;
-            const int s = it % S;
-            const uint32_t ph = (it / S) & 1;
-            if (rb != cur_rb) {
-                // the previous row block's last partial first, then finish it
-                if (have_prev) {
-                    if (!fold(prev_scale)) { ok = false; break; }
-                    have_prev = false;
-                }
-                if (cur_rb >= 0 && !flush(cur_rb)) { ok = false; break; }
-                cur_rb = rb;
-                first_ks = ks;
-#pragma unroll
-                for (int i = 0; i < NN; ++i) acc[i] = 0.0f;
-            }
-            last_ks = ks;
-            const bool mine = 2 * ks + h < G;  // this unit has a group for this warpgroup
-            if (!warp_wait(smem_u32(&sh->full[s]), ph, abort_flag, status)) { ok = false; break; }
-            const uint8_t *st = ring + s * C::kBytes;
-            float sc = 0.0f;
-            if (mine) {
-                const float *ss = reinterpret_cast<const float *>(st + C::kSZ);
-                const float *zz = ss + 2 * kUnitRows;
-                sc = ss[2 * r + h];
-                uint32_t zb, zq;
-                zero_bias<XT>(zeros ? zz[2 * r + h] : 8.0f, zb, zq);
-                // this row's 128 codes of group h: four swizzled 16-byte chunks
-                uint32_t wv[16];
-#pragma unroll
-                for (int cch = 0; cch < 4; ++cch) {
-                    const uint4 v =
-                        *reinterpret_cast<const uint4 *>(st + r * 128 + (((4 * h + cch) ^ swz) << 4));
-                    wv[4 * cch] = v.x;
-                    wv[4 * cch + 1] = v.y;
-                    wv[4 * cch + 2] = v.z;
-                    wv[4 * cch + 3] = v.w;
-                }
-                const uint32_t b = n_a & 1, pb = (n_a >> 1) & 1;
-                if (!warp_wait(smem_u32(&sh->afree[h][b]), pb ^ 1, abort_flag, status)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t ta = tmem + lanebase + (uint32_t)((2 * h + b) * kAColsPerGroup);
-#pragma unroll
-                for (int kb = 0; kb < 8; ++kb) {
-                    uint32_t a[8];
-                    dequant_word<XT>(wv[2 * kb], zb, zq, a);
-                    dequant_word<XT>(wv[2 * kb + 1], zb, zq, a + 4);
-                    tmem_st8(ta + 8 * kb, a);
-                }
-                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-                tc_fence_before();
-                mbar_arrive(smem_u32(&sh->afull[h][b]));
-                ++n_a;
-            }
-            // fold the previous unit's partial while this unit's MMAs run
-            if (have_prev) {
-                if (!fold(prev_scale)) { ok = false; break; }
-                have_prev = false;
-            }
-            if (mine) {
-                prev_scale = sc;
-                have_prev = true;
-            }
-            if (++ks == wk.KS) {
-                ks = 0;
-                ++rb;
-            }
         }
-        if (ok && have_prev) ok = fold(prev_scale);
-        if (ok && cur_rb >= 0) ok = flush(cur_rb);
-        if (ok && h == 0) finish_partials();
     }
+
 
     tc_fence_before();
     __syncthreads();
