@@ -26,6 +26,7 @@ scaling); no data-path collective.  Time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -45,6 +46,13 @@ import synth  # noqa: E402
 
 METRIC = "W4A16 g128 dequant-GEMM TB/s (decode) & TFLOPS (prefill) vs B200 roofline"
 GROUP = 128
+
+# DRAM traffic of one decode launch (M=1, K=4096, N=12288: the dominant
+# kernel of the step) from one ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum; profiles/decode_kernel_m1_k4096_n12288.md), valid
+# only for the kernel source it was taken on: reported as null once that
+# source has changed.
+DECODE_TRAFFIC = {"bytes": 28389888, "source_sha256_16": "16eb1aeea6e5e546"}
 
 
 # ---------------------------------------------------------------------------- helpers
@@ -310,9 +318,13 @@ def run_ours(args, ws_, rank, local):
         b = decode_bytes(1, K, N, c["sym"])
         per_layer.append({"N": N, "us": kms * 1e3, "bytes": b, "gbs": b / (kms * 1e-3) / 1e9})
     dom = max(per_layer, key=lambda d: d["us"])
+    src = os.path.join(ROOT, "weight_only_int4_pack_b200", "csrc", "w4_decode.cu")
+    cur = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] if os.path.exists(src) else ""
+    traffic = DECODE_TRAFFIC["bytes"] if (cur == DECODE_TRAFFIC["source_sha256_16"]
+                                          and dom["N"] == 12288) else None
     roof = {"bound": "hbm", "kernel": "decode_kernel (w4a16_gemm, M=1)",
             "achieved": round(dom["gbs"], 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-            "frac": round(dom["gbs"] / pk["hbm_gbs"], 4), "traffic": None,
+            "frac": round(dom["gbs"] / pk["hbm_gbs"], 4), "traffic": traffic,
             "peak_source": pk["source"], "bytes_per_launch": dom["bytes"],
             "launch_us": round(dom["us"], 3), "per_layer": per_layer}
 
