@@ -159,6 +159,20 @@ int w4a16_gemm_noalloc(const void *X, int xt, int64_t M, const uint8_t *packed,
 int w4_device_status(int reset);
 
 /*
+ * w4_selftest_wait_timeout -- failure-detection self-test (the pages have no
+ * counterpart).  Enqueues on `stream` one small kernel whose only mbarrier
+ * wait can never complete (nothing arrives on the barrier).  The wait is
+ * bounded by timeout_us microseconds (1 .. 1000000), exactly as every wait
+ * of the library's kernels is bounded by its own limit: when it runs out the
+ * kernel sets the device status word and returns, and the CUDA context stays
+ * usable.  A caller (or a test) checks the mechanism with
+ * w4_device_status(1) == W4_ERR_TIMEOUT afterwards.
+ * Returns W4_OK once the kernel is enqueued, W4_ERR_INVALID_ARG for a
+ * timeout out of range, W4_ERR_CUDA if the launch fails.
+ */
+int w4_selftest_wait_timeout(unsigned timeout_us, void *stream);
+
+/*
  * w4_last_error -- text describing the most recent failure on the calling
  * thread: which check or which CUDA call failed, and why ("" if none yet).
  * Thread-local storage owned by the library, valid until the thread's next

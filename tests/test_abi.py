@@ -121,3 +121,10 @@ def test_product_package_does_not_reach_the_oracle():
             src = open(os.path.join(dirpath, fn)).read()
             assert "import oracle" not in src and "from oracle" not in src, fn
             assert "w4ref" not in src and "libw4ref" not in src, fn
+
+
+def test_selftest_argument_check(lib):
+    """The timeout range is checked on the host before any CUDA call."""
+    for bad in (0, 1000001):
+        assert lib.w4_selftest_wait_timeout(bad, None) == w4.W4_ERR_INVALID_ARG
+        assert b"timeout_us" in lib.w4_last_error()

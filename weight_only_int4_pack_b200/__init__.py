@@ -25,7 +25,7 @@ import torch
 __all__ = [
     "W4Error", "load", "lib_path", "w4_quantize", "w4_quantize_into", "w4a16_workspace_bytes",
     "w4a16_gemm", "w4a16_gemm_into", "w4_status_string", "w4_device_status", "w4_abi_version",
-    "w4_last_error", "w4a16_gemm_noalloc",
+    "w4_last_error", "w4a16_gemm_noalloc", "w4_selftest_wait_timeout",
     "Workspace", "W4_OK", "W4_ERR_INVALID_ARG", "W4_ERR_UNSUPPORTED", "W4_ERR_CUDA",
     "W4_ERR_TIMEOUT", "W4_F16", "W4_BF16",
 ]
@@ -73,6 +73,8 @@ def load() -> ctypes.CDLL:
     lib.w4_abi_version.restype = I
     lib.w4a16_gemm_noalloc.argtypes = [P, I, I64, P, P, P, I64, I64, I, P, P]
     lib.w4a16_gemm_noalloc.restype = I
+    lib.w4_selftest_wait_timeout.argtypes = [ctypes.c_uint, P]
+    lib.w4_selftest_wait_timeout.restype = I
     lib.w4_last_error.argtypes = []
     lib.w4_last_error.restype = ctypes.c_char_p
     _lib = lib
@@ -125,6 +127,15 @@ def w4_abi_version() -> int:
 def w4_device_status(reset: bool = True) -> int:
     """Status word set by kernels whose bounded waits ran out (synchronizes)."""
     return int(load().w4_device_status(int(bool(reset))))
+
+
+def w4_selftest_wait_timeout(timeout_us: int = 1000, stream=None) -> None:
+    """Enqueue the failure-detection self-test: a kernel whose only wait can
+    never complete times out after `timeout_us` and sets the device status
+    word (read it with w4_device_status)."""
+    st = load().w4_selftest_wait_timeout(int(timeout_us), _stream(stream))
+    if st != W4_OK:
+        raise W4Error("w4_selftest_wait_timeout", st)
 
 
 def w4_quantize_into(W, packed, scales, zeros, group=128, sym=True, col_scale=None, stream=None):

@@ -22,6 +22,39 @@ unsigned *g_status_ptr[kMaxDevices] = {};
 
 thread_local char g_last_error[320] = "";
 
+// One warp; lane 0 waits on an mbarrier that nothing arrives on, bounded by
+// limit_ns of the global timer, then records the timeout in the status word.
+__global__ void selftest_wait_kernel(unsigned long long limit_ns, unsigned *status) {
+    __shared__ uint64_t bar;
+    const uint32_t b = static_cast<uint32_t>(__cvta_generic_to_shared(&bar));
+    if (threadIdx.x == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(b));
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+    if (threadIdx.x == 0) {
+        unsigned long long t0, t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+        while (true) {
+            uint32_t ok;
+            asm volatile(
+                "{\n\t.reg .pred p;\n\t"
+                "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\n\t"
+                "selp.u32 %0, 1, 0, p;\n\t}"
+                : "=r"(ok)
+                : "r"(b)
+                : "memory");
+            if (ok) break;  // cannot happen: nothing arrives
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+            if (t - t0 > limit_ns) {
+                atomicOr(status, 1u);
+                break;
+            }
+        }
+    }
+    __syncwarp();
+}
+
 bool valid_dtype(int t) { return t == W4_F16 || t == W4_BF16; }
 
 int reject(int status, const char *fn, const char *why) { return w4::set_error(status, fn, why); }
@@ -206,6 +239,19 @@ int w4a16_gemm(const void *X, int xt, int64_t M, const uint8_t *packed, const fl
                size_t workspace_bytes, void *stream) {
     return gemm_impl(X, xt, M, packed, scales, zeros, K, N, group, Y, workspace, workspace_bytes,
                      stream);
+}
+
+int w4_selftest_wait_timeout(unsigned timeout_us, void *stream) {
+    if (timeout_us < 1 || timeout_us > 1000000)
+        return w4::set_error(W4_ERR_INVALID_ARG, "w4_selftest_wait_timeout",
+                             "timeout_us must be 1 .. 1000000");
+    unsigned *status = w4::device_status_ptr();
+    if (!status) return W4_ERR_CUDA;
+    selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<unsigned long long>(timeout_us) * 1000ull, status);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return w4::cuda_fail("selftest_wait_kernel launch", e);
+    return W4_OK;
 }
 
 int w4_device_status(int reset) {
