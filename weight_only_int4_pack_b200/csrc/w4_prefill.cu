@@ -18,22 +18,28 @@
 // fp32 partial in TMEM, and the epilogue adds scale * partial into fp32
 // registers.  No weight is rounded to 16 bits.
 //
-// Warp roles (320 threads):
-//   warp 0      TMA producer: X tile (256 x 64, 128B swizzle) and the packed
-//               codes of 128 rows x 64 k into a 4-stage shared-memory ring.
-//   warp 1      TMEM allocator and MMA issuer (one thread): 4 x
-//               tcgen05.mma.kind::f16 (128 x 256 x 16) per stage into the
-//               group's partial buffer P[b] (2 x 256 TMEM columns).
-//   warps 2..9  math: (a) dequantize each stage's codes into the bf16/fp16
-//               A tile (128B-swizzled K-major, the layout the MMA descriptor
-//               names) and (b) per group, read P[b] with tcgen05.ld and
-//               accumulate acc += scale * P into registers (two warps per
-//               TMEM lane quarter, 128 columns each).  After the last group
-//               of a tile they round acc to the output dtype and store Y.
+// Warp roles (512 threads, four warpgroups):
+//   warp 0       TMA producer: X tile (256 x 64, 128B swizzle) and the packed
+//                codes of 128 rows x 64 k into a 4-stage shared-memory ring.
+//   warp 1       TMEM allocator and MMA issuer (one thread): 4 x
+//                tcgen05.mma.kind::f16 (128 x 256 x 16) per stage into the
+//                group's partial buffer P[b] (2 x 256 TMEM columns).
+//   warps 2, 3   no role (they only give their registers back).
+//   warps 4..7   dequantize: thread t writes row t of each stage's A tile
+//                (the bf16/fp16 values of 64 k, 128B-swizzled K-major, the
+//                layout the MMA descriptor names), as soon as the stage's
+//                codes have landed -- up to the whole ring ahead of the MMAs.
+//   warps 8..15  fold: per group, read P[b] with tcgen05.ld and accumulate
+//                acc += scale * P into registers (two warps per TMEM lane
+//                quarter, 128 columns each).  After the last group of a tile
+//                they round acc to the output dtype and store Y.
+// Dequantization and folding are separate warps so that the A tile of group
+// g + 2 never waits for the fold of group g.
 //
-// Registers: each SM sub-partition has 16K registers and this 10-warp CTA puts
-// three warps on two of them, so a thread may hold at most 168 registers
-// (the math warps keep 128 fp32 accumulators).
+// Registers: the CTA is launched with 128 a thread (512 x 128 = the SM's 64K);
+// warpgroups 0 and 1 give back to 88 and warpgroups 2 and 3 (the fold warps,
+// which keep 128 fp32 accumulators) take 168: 2 x 128 x 88 + 2 x 128 x 168 =
+// 65536, exactly what the CTA was launched with.
 //
 // Every wait on an mbarrier is bounded (kWaitNs); a wait that runs out sets
 // the library's device status word to W4_ERR_TIMEOUT and a shared abort
@@ -57,8 +63,10 @@ constexpr int kBN = 256;       // activation rows per tile (MMA N)
 constexpr int kBK = 64;        // k per pipeline stage (one 128-byte swizzle row of 16-bit)
 constexpr int kStages = 4;
 constexpr int kGroup = 128;
-constexpr int kMathWarps = 8;
-constexpr int kThreads = 64 + 32 * kMathWarps;  // 320
+constexpr int kFoldWarps = 8;
+constexpr int kThreads = 512;
+constexpr int kDequantWarp0 = 4;
+constexpr int kFoldWarp0 = 8;
 constexpr int kTmemCols = 512;                  // 2 partial buffers x 256 columns
 
 constexpr int kXTileBytes = kBN * kBK * 2;      // 32 KB
@@ -258,13 +266,13 @@ struct Smem {
 };
 
 // Dequantizes the two stages of group g of the current tile (stage counter
-// base `it`) for this thread's A-tile row dr, k half dkh: waits for the codes,
-// writes 4 swizzled 16-byte chunks per stage, fences them for the tensor
-// core and arrives on the stage's A-ready barrier.
+// base `it`) for this thread's A-tile row dr: waits for the codes, writes the
+// row's 8 swizzled 16-byte chunks per stage, fences them for the tensor core
+// and arrives on the stage's A-ready barrier.
 template <int XT>
 __device__ __forceinline__ bool dequant_group(int g, uint32_t it, int n_d, int G,
                                               const float *__restrict__ zeros, const uint8_t *cs,
-                                              uint8_t *as, int dr, int dkh, Smem *sm,
+                                              uint8_t *as, int dr, Smem *sm,
                                               volatile int *abort_flag, unsigned *status) {
     const float z = zeros ? __ldg(zeros + (int64_t)n_d * G + g) : 8.0f;
     uint32_t zb, zq;
@@ -277,13 +285,14 @@ __device__ __forceinline__ bool dequant_group(int g, uint32_t it, int n_d, int G
         // warp-uniform outcome: the warp either goes on together or leaves together
         if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm->full[s]), ph, abort_flag, status)))
             return false;
-        const uint4 w =
-            *reinterpret_cast<const uint4 *>(cs + s * kCodeTileBytes + dr * (kBK / 2) + dkh * 16);
+        const uint8_t *crow = cs + s * kCodeTileBytes + dr * (kBK / 2);
+        const uint4 w0 = *reinterpret_cast<const uint4 *>(crow);
+        const uint4 w1 = *reinterpret_cast<const uint4 *>(crow + 16);
         uint8_t *arow = as + s * kATileBytes + dr * 128;
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        const uint32_t ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            const int chunk = (dkh * 4 + jj) ^ (dr & 7);
+        for (int jj = 0; jj < 8; ++jj) {
+            const int chunk = jj ^ (dr & 7);
             *reinterpret_cast<uint4 *>(arow + chunk * 16) = dequant_word<XT>(ws[jj], zb, zq);
         }
         fence_proxy_async();
@@ -293,7 +302,7 @@ __device__ __forceinline__ bool dequant_group(int g, uint32_t it, int n_d, int G
 }
 
 template <int XT>
-__global__ void __maxnreg__(168)
+__global__ void __launch_bounds__(kThreads, 1)
 prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                const float *__restrict__ scales, const float *__restrict__ zeros, int M, int N,
                int K, void *__restrict__ Y, unsigned *__restrict__ status) {
@@ -319,11 +328,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
         for (int s = 0; s < kStages; ++s) {
             mbar_init(smem_u32(&sm->full[s]), 1);
             mbar_init(smem_u32(&sm->empty[s]), 1);
-            mbar_init(smem_u32(&sm->aready[s]), 32 * kMathWarps);
+            mbar_init(smem_u32(&sm->aready[s]), kBM);  // one dequant thread per row
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&sm->pfull[b]), 1);
-            mbar_init(smem_u32(&sm->pempty[b]), 32 * kMathWarps);
+            mbar_init(smem_u32(&sm->pempty[b]), 32 * kFoldWarps);
         }
         sm->abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -339,7 +348,11 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     tc_fence_after();
     const uint32_t tmem = sm->tmem_base;
 
-    if (warp == 0) {
+    // Register split (see the header): each warpgroup's branch starts with its
+    // setmaxnreg, executed by all four of its warps.
+    if (warp < 4) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 88;" ::: "memory");
+      if (warp == 0) {
         // ---------------- TMA producer ----------------
         if (lane == 0) {
             uint32_t it = 0;
@@ -369,7 +382,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             }
         }
         __syncwarp();  // the whole warp reconverges before the CTA barrier
-    } else if (warp == 1) {
+      } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
             constexpr uint32_t idesc = instr_desc<XT>();
@@ -417,48 +430,40 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             }
         }
         __syncwarp();  // the whole warp reconverges before the CTA barrier
+      }
+    } else if (warp < kFoldWarp0) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 88;" ::: "memory");
+        // ---------------- dequantize: thread = A-tile row ----------------
+        const int dr = threadIdx.x - 32 * kDequantWarp0;  // 0..127
+        uint32_t it = 0;
+        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+            const int nt = tile % n_tiles;
+            const int n_d = min(nt * kBM + dr, N - 1);  // clamped: rows past N are never stored
+            bool ok = true;
+            for (int g = 0; g < G && ok; ++g)
+                ok = dequant_group<XT>(g, it, n_d, G, zeros, cs, as, dr, sm, abort_flag, status);
+            if (!ok) break;
+            it += (uint32_t)kstages_per_tile;
+        }
     } else {
-        // ---------------- math warps: dequant + epilogue ----------------
-        const int mw = warp - 2;             // 0..7
-        const int q = warp & 3;              // TMEM lane quarter this warp may access
-        const int colhalf = mw >> 2;         // 0: columns 0..127, 1: 128..255
-        const int mt_idx = threadIdx.x - 64; // 0..255
-        // dequant role: row r of the A tile, k half kh (32 k = 4 words)
-        const int dr = mt_idx & (kBM - 1);
-        const int dkh = mt_idx >> 7;
-        // epilogue role: TMEM lane (= weight row of the tile)
-        const int er = 32 * q + lane;
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 168;" ::: "memory");
+        // ---------------- fold + epilogue ----------------
+        const int fw = warp - kFoldWarp0;  // 0..7
+        const int q = warp & 3;            // TMEM lane quarter this warp may access
+        const int colhalf = fw >> 2;       // 0: columns 0..127, 1: 128..255
+        const int er = 32 * q + lane;      // TMEM lane = weight row of the tile
 
         float acc[128];
-        uint32_t it = 0, gc = 0;
+        uint32_t gc = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
             const int nt = tile % n_tiles, mt = tile / n_tiles;
-            const int n_d = min(nt * kBM + dr, N - 1);  // dequant row (clamped)
-            const int n_e = nt * kBM + er;              // epilogue row
+            const int n_e = nt * kBM + er;
             const int n_ec = min(n_e, N - 1);
 #pragma unroll
             for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
-
-            // Stay at most one group ahead with the dequantization: the ring holds
-            // kStages = 2 groups of stages, and a stage can only be refilled once
-            // the MMAs of the group before it have run.
-            int next_dq_group = 0;
-            if (!dequant_group<XT>(0, it, n_d, G, zeros, cs, as, dr, dkh, sm, abort_flag, status)) {
-                ok = false;
-                break;
-            }
-            next_dq_group = 1;
             float s_next = __ldg(scales + (int64_t)n_ec * G + 0);
             for (int g = 0; g < G; ++g, ++gc) {
-                if (next_dq_group < G) {
-                    if (!dequant_group<XT>(next_dq_group, it, n_d, G, zeros, cs, as, dr, dkh, sm,
-                                           abort_flag, status)) {
-                        ok = false;
-                        break;
-                    }
-                    ++next_dq_group;
-                }
                 const float sg = s_next;
                 if (g + 1 < G) s_next = __ldg(scales + (int64_t)n_ec * G + g + 1);
                 const int b = gc & 1;
@@ -484,7 +489,6 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                 mbar_arrive(smem_u32(&sm->pempty[b]));
             }
             if (!ok) break;
-            it += (uint32_t)kstages_per_tile;
             // store this thread's row n_e for its 128 columns m
             if (n_e < N) {
                 const int m0 = mt * kBN + colhalf * 128;
