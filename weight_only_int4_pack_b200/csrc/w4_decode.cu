@@ -794,7 +794,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         // Arrives on the counters of the split row blocks this warp stored; the
         // last warp to arrive on one adds its partials in CTA order.
         if (ok && p == 0 && pend0 >= 0) {
-            __threadfence();
+            // One acquire-release atomic per split row block: it orders this
+            // warp's partial stores (made by every lane, joined by __syncwarp)
+            // before the arrival, and the last arriver's loads of the other
+            // CTAs' partials after it.
             __syncwarp();
             for (int pi = 0; pi < 2; ++pi) {
                 const int prb = pi == 0 ? pend0 : pend1;
@@ -802,10 +805,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                 const int cf = owner(wk, prb * wk.KS), cl = owner(wk, (prb + 1) * wk.KS - 1);
                 unsigned *cnt = counters + prb * 8 + q;
                 unsigned prev = 0;
-                if (lane == 0) prev = atomicAdd(cnt, 1u);
+                if (lane == 0)
+                    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                                 : "=r"(prev)
+                                 : "l"(cnt)
+                                 : "memory");
                 prev = __shfl_sync(0xffffffffu, prev, 0);
                 if (prev != (unsigned)(cl - cf)) continue;
-                __threadfence();
+                __syncwarp();
                 const int n = prb * kUnitRows + r;
                 if (n < N) {
                     for (int m = 0; m < M; ++m) {

@@ -476,14 +476,18 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                 tc_fence_after();
                 const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16) +
                                        static_cast<uint32_t>(b * kBN + colhalf * 128);
+                // two 16-column loads in flight per wait
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t r[16];
-                    tmem_ld16(taddr + 16 * c, r);
+                for (int c = 0; c < 8; c += 2) {
+                    uint32_t r0[16], r1[16];
+                    tmem_ld16(taddr + 16 * c, r0);
+                    tmem_ld16(taddr + 16 * (c + 1), r1);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        acc[16 * c + i] = fmaf(sg, __uint_as_float(r[i]), acc[16 * c + i]);
+                    for (int i = 0; i < 16; ++i) {
+                        acc[16 * c + i] = fmaf(sg, __uint_as_float(r0[i]), acc[16 * c + i]);
+                        acc[16 * (c + 1) + i] = fmaf(sg, __uint_as_float(r1[i]), acc[16 * (c + 1) + i]);
+                    }
                 }
                 tc_fence_before();
                 mbar_arrive(smem_u32(&sm->pempty[b]));
