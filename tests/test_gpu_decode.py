@@ -130,3 +130,26 @@ def test_quantize_then_gemm_on_device():
     p, s, z = oracle_quantize(W, 128, False)
     assert np.array_equal(packed.cpu().numpy(), p)
     check_y(Y, oracle_linear(X, p, s, z, K), "device path")
+
+
+def test_back_to_back_launches_overlap():
+    """Layers launched one after another with no synchronization in between:
+    with programmatic dependent launch a launch's CTAs start (and stream
+    their weights) while the previous launch's CTAs finish on the same SMs,
+    and wait for its tensor memory.  Every output must still match."""
+    shapes = [(1, 1000, 1024), (1, 4096, 4096), (3, 2000, 2048), (1, 12288, 4096), (16, 700, 1024)]
+    cases = []
+    for i, (M, N, K) in enumerate(shapes):
+        W = synth.weights(N, K, 0.02, 900 + i)
+        X = synth.activations(M, K, 900 + i)
+        packed, scales, zeros = oracle_quantize(W, 128, i % 2 == 0)
+        pd, sd, zd = to_dev(packed, scales, zeros)
+        cases.append((X, X.to(DEV), packed, scales, zeros, pd, sd, zd, K))
+    outs = []
+    for rep in range(3):
+        outs.append([w4.w4a16_gemm(Xd, pd, sd, zd) for (_, Xd, _, _, _, pd, sd, zd, _) in cases])
+    torch.cuda.synchronize()
+    for rep in range(3):
+        for (X, _, packed, scales, zeros, _, _, _, K), Y in zip(cases, outs[rep]):
+            check_y(Y, oracle_linear(X, packed, scales, zeros, K, 128), f"back-to-back rep {rep}")
+    assert w4.w4_device_status() == w4.W4_OK
