@@ -638,7 +638,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
 #pragma unroll
         for (int i = 0; i < NN; ++i) acc[i] = 0.0f;
         int cur_rb = -1;      // row block the accumulators belong to
-        int pend0 = -1, pend1 = -1;  // split row blocks stored (p == 0)
+        int pend0 = -1, pend1 = -1;
+        unsigned prev0 = 0, prev1 = 0;  // their counters before this warp's arrival (lane 0)  // split row blocks stored (p == 0)
         uint32_t nflush = 0;  // row blocks flushed (xfull / xfree parity)
         bool ok = true;
 
@@ -673,10 +674,25 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
 #pragma unroll
             for (int m = 0; m < NN; ++m)
                 if (m < M) dst[m] = acc[m];
-            if (pend0 < 0)
+            // Arrive on the row block's (row block, lane quarter) counter at
+            // once: one acquire-release atomic orders this warp's partial
+            // stores (every lane's, joined by __syncwarp) before the arrival;
+            // its result (was this the last arrival?) is only looked at after
+            // the CTA's last unit, so the round trip overlaps the work.
+            __syncwarp();
+            unsigned prev = 0;
+            if (lane == 0)
+                asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                             : "=r"(prev)
+                             : "l"(counters + rb * 8 + q)
+                             : "memory");
+            if (pend0 < 0) {
                 pend0 = rb;
-            else
+                prev0 = prev;
+            } else {
                 pend1 = rb;
+                prev1 = prev;
+            }
             return true;
         };
 
@@ -793,24 +809,15 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         if (ok && cur_rb >= 0) ok = flush(cur_rb);
         // Arrives on the counters of the split row blocks this warp stored; the
         // last warp to arrive on one adds its partials in CTA order.
+        // The last warp to arrive on a split row block's counter adds the
+        // partials in CTA order, writes Y and re-arms the counter.
         if (ok && p == 0 && pend0 >= 0) {
-            // One acquire-release atomic per split row block: it orders this
-            // warp's partial stores (made by every lane, joined by __syncwarp)
-            // before the arrival, and the last arriver's loads of the other
-            // CTAs' partials after it.
-            __syncwarp();
             for (int pi = 0; pi < 2; ++pi) {
                 const int prb = pi == 0 ? pend0 : pend1;
                 if (prb < 0) break;
                 const int cf = owner(wk, prb * wk.KS), cl = owner(wk, (prb + 1) * wk.KS - 1);
                 unsigned *cnt = counters + prb * 8 + q;
-                unsigned prev = 0;
-                if (lane == 0)
-                    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
-                                 : "=r"(prev)
-                                 : "l"(cnt)
-                                 : "memory");
-                prev = __shfl_sync(0xffffffffu, prev, 0);
+                const unsigned prev = __shfl_sync(0xffffffffu, pi == 0 ? prev0 : prev1, 0);
                 if (prev != (unsigned)(cl - cf)) continue;
                 __syncwarp();
                 const int n = prb * kUnitRows + r;
