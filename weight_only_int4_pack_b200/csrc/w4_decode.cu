@@ -429,7 +429,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     const int nu = u1 - u0;
     const int G = wk.G;
 
+    // The packed weights are inputs no earlier kernel writes: thread 0 (the
+    // producer's TMA lane) requests the codes of the CTA's first two units as
+    // soon as the barriers exist, before anything else of the prologue.
+    const int early = min(2, min(S, nu));
     if (threadIdx.x == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_w)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
         for (int s = 0; s < S; ++s) {
             mbar_init(smem_u32(&sh->full[s]), 1 + 32);  // TMA arrive_tx + 32 cp.async arrivals
             mbar_init(smem_u32(&sh->empty[s]), 1);
@@ -444,6 +450,17 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         }
         sh->abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        int rb = u0 / wk.KS, ks = u0 - (u0 / wk.KS) * wk.KS;
+        for (int it = 0; it < early; ++it) {
+            const uint32_t fb = smem_u32(&sh->full[it]);
+            mbar_arrive_tx(fb, C::kTmaBytes);
+            tma_load_2d(smem_u32(ring + it * C::kBytes), &tmap_w, ks * (kUnitK / 2), rb * kUnitRows,
+                        fb);
+            if (++ks == wk.KS) {
+                ks = 0;
+                ++rb;
+            }
+        }
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -489,23 +506,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         };
         // (rb, ks): row block and k step of the next unit to issue
         int rb = u0 / wk.KS, ks = u0 - (u0 / wk.KS) * wk.KS;
-        // The packed weights are inputs no earlier kernel writes: the codes of
-        // the first two units are requested before waiting for the preceding
-        // kernel; the X slices, zero points and scales of the first units go
-        // out before the rest of the first ring, so that unit 0 lands early.
+        // The codes of the first `early` units went out in the prologue; the
+        // X slices and zero points of the first units go out before the rest
+        // of the first ring, so that unit 0 lands early.
         const int pre = min(S, nu);
-        const int early = min(2, pre);
-        if (lane == 0) {
-            int rb2 = rb, ks2 = ks;
-            for (int it = 0; it < early; ++it) {
-                issue_w(rb2, ks2, ring + it * C::kBytes, smem_u32(&sh->full[it]));
-                if (++ks2 == wk.KS) {
-                    ks2 = 0;
-                    ++rb2;
-                }
-            }
-        }
-        __syncwarp();
         asm volatile("griddepcontrol.wait;" ::: "memory");
         for (int it = 0; it < pre; ++it) {
             uint8_t *st = ring + it * C::kBytes;
