@@ -170,7 +170,8 @@ def ranges(K, N, sms=148):
 
 
 @pytest.mark.parametrize("K,N", [(4096, 4096), (4096, 11008), (4096, 12288), (8192, 28672),
-                                 (384, 1000), (640, 300), (128, 100), (11008, 4096)])
+                                 (384, 1000), (640, 300), (128, 100), (11008, 4096),
+                                 (256, 160000), (128, 270000), (384, 151553)])
 @pytest.mark.parametrize("R,S", [(3, 7), (2, 5)])
 def test_no_deadlock(K, N, R, S):
     KS, rs = ranges(K, N)

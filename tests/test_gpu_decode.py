@@ -81,6 +81,15 @@ def test_shapes(N, K, M):
     case(M, N, K, True, "f16", N * 7 + K + M, x_salient=0.01)
 
 
+@pytest.mark.parametrize("M,N,K", [(1, 160000, 256), (2, 270000, 128), (5, 151553, 384)])
+def test_whole_row_block_ranges(M, N, K):
+    """Many row blocks per CTA (>= 8 per SM) or more row blocks than the
+    workspace counter area holds: every CTA takes whole row blocks, no K is
+    split across CTAs and no workspace is needed."""
+    assert w4.w4a16_workspace_bytes(M, K, N) == 0
+    case(M, N, K, False, "f16", N + K + M, x_salient=0.01)
+
+
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 def test_symmetric_without_zero_points(dtype):
     case(4, 96, 512, True, dtype, 5, pass_zeros=False)
