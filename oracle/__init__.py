@@ -10,7 +10,8 @@ Sources followed (see ``w4ref.c`` for the step-by-step citations):
 "LLM quantization methods: principles and implementation"
 (zhiyuanblog.org/blog/llm-quantization) §2.2-§2.3 and §4.2, and
 "PTQ weight quantization: from GPTQ to AWQ" (jonathanding.github.io),
-sections "Round-to-Nearest" and "AWQ".
+sections "Round-to-Nearest" and "AWQ" (the AWQ scale search of §4.2 is
+``awq_search``).
 """
 from __future__ import annotations
 
@@ -66,6 +67,10 @@ def _load():
         lib.w4ref_f16_to_f64.restype = ctypes.c_double
         lib.w4ref_bf16_to_f64.argtypes = [ctypes.c_uint16]
         lib.w4ref_bf16_to_f64.restype = ctypes.c_double
+        lib.w4ref_round16.argtypes = [ctypes.c_double, I]
+        lib.w4ref_round16.restype = ctypes.c_double
+        lib.w4ref_awq_search.argtypes = [P, P, I, L, L, L, L, I, P, L, P, P, P]
+        lib.w4ref_awq_search.restype = I
         lib.w4ref_threads.argtypes = []
         lib.w4ref_threads.restype = I
         lib.w4ref_set_threads.argtypes = [I]
@@ -178,3 +183,32 @@ def f16_to_f64(h: int) -> float:
 
 def bf16_to_f64(h: int) -> float:
     return float(_load().w4ref_bf16_to_f64(h))
+
+
+def round16(v: float, dtype: int) -> float:
+    """Nearest fp16 / bf16 value to v (ties to even), as a float; +-inf on overflow."""
+    return float(_load().w4ref_round16(float(v), dtype))
+
+
+def awq_search(W, X, dtype: int, group: int, sym: bool, alphas):
+    """AWQ grid search over alpha for one layer.
+
+    W [N][K] and calibration activations X [Mc][K] (uint16 bits or float16).
+    Returns (err fp64 [n_alpha], s fp32 [n_alpha][K], best index) where
+    err[t] = || Q(W * s_t)(X / s_t) - W X ||_F^2 and s_t = (a / w)^alphas[t].
+    """
+    W = _bits16(W)
+    X = _bits16(X)
+    N, K = W.shape
+    Mc, K2 = X.shape
+    assert K2 == K
+    alphas = np.ascontiguousarray(alphas, dtype=np.float32).ravel()
+    err = np.full(alphas.shape[0], np.nan, np.float64)
+    s_all = np.zeros((alphas.shape[0], K), np.float32)
+    best = ctypes.c_long(-1)
+    st = _load().w4ref_awq_search(_ptr(W), _ptr(X), dtype, Mc, K, N, group, int(bool(sym)),
+                                  _ptr(alphas), alphas.shape[0], _ptr(err), _ptr(s_all),
+                                  ctypes.byref(best))
+    if st != OK:
+        raise OracleError(f"w4ref_awq_search status {st}")
+    return err, s_all, int(best.value)

@@ -18,7 +18,9 @@
  *              dimension is cut into groups of g (e.g. 128) with one scale each,
  *              and in_features must be a multiple of g.
  *         §4.2 AWQ: W is multiplied column-wise by a per-input-channel factor s
- *              before the per-group quantizer runs.
+ *              before the per-group quantizer runs; s = (a/w)^alpha from the
+ *              mean magnitudes of activations and weights, alpha grid-searched
+ *              to minimise the layer's output error.
  *   [PTQ] "PTQ weight quantization: from GPTQ to AWQ" (jonathanding.github.io),
  *         section "Round-to-Nearest": every weight is rounded on its own to the
  *         nearest level; section "AWQ": XW = (X diag(s)^-1)(diag(s) W).
@@ -49,6 +51,7 @@
 #include <fenv.h>
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #define W4REF_OK 0
@@ -293,3 +296,164 @@ void w4ref_set_threads(int n) { omp_set_num_threads(n); }
 int w4ref_threads(void) { return 1; }
 void w4ref_set_threads(int n) { (void)n; }
 #endif
+
+/* ---- AWQ per-input-channel scale search ------------------------------------------------ */
+
+/*
+ * Nearest binary16 (dtype F16) or bfloat16 (dtype BF16) value to v, ties to
+ * even, returned as a double; from the formats' definitions: p significant
+ * bits (11 / 8), smallest normal exponent emin (-14 / -126), below which the
+ * spacing stays 2^(emin - p + 1) (subnormals), and largest finite value
+ * (65504 / (2 - 2^-7) * 2^127).  A magnitude that rounds above it is +-inf.
+ */
+double w4ref_round16(double v, int dtype)
+{
+    if (v == 0.0 || isnan(v) || isinf(v)) return v;
+    const int p = dtype == DT_BF16 ? 8 : 11;
+    const int emin = dtype == DT_BF16 ? -126 : -14;
+    const double maxv = dtype == DT_BF16 ? ldexp(255.0, 120) : 65504.0;
+    int e;
+    frexp(v, &e); /* |v| = f * 2^e with f in [0.5, 1): the leading bit is worth 2^(e-1) */
+    int lead = e - 1;
+    if (lead < emin) lead = emin;
+    const int q = lead - (p - 1); /* exponent of one unit in the last place */
+    const double r = ldexp(nearbyint(ldexp(v, -q)), q);
+    if (fabs(r) > maxv) return copysign(INFINITY, v);
+    return r;
+}
+
+/*
+ * AWQ scale search for one linear layer.
+ *   [LQ] §4.2: find the per-input-channel factor s that minimises
+ *        || Q(W * s) (X / s) - W X ||; its code form takes, per input
+ *        channel j, the activation importance a_j = mean_i |X_ij| and the
+ *        weight magnitude w_j = mean_n |W_nj|, forms s_j = (a_j / w_j)^alpha,
+ *        scales the columns of W by s before the per-group quantizer, and at
+ *        inference divides the activations by s; alpha in [0, 1] is picked by
+ *        a grid search.
+ *   [PTQ] section "AWQ": the same identity XW = (X diag(s)^-1)(diag(s) W).
+ *
+ * Inputs: W [N][K] and the calibration activations X [Mc][K], both 16-bit
+ * bit patterns of `dtype`; alphas [n_alpha].
+ * Outputs: err [n_alpha]; s_all (nullable) [n_alpha][K] fp32; *best.
+ *
+ * Readings where the pages leave a step open:
+ *   - a_j and w_j are fp64 sums in index order, divided by the count in
+ *     fp64 and rounded once to fp32;
+ *   - s_j = fl32(pow(a_j / w_j, alpha)) with the ratio and pow in fp64, and
+ *     s_j = 1 for a channel whose a_j or w_j is 0 (no evidence either way);
+ *   - Q is the per-group RTN quantizer above with col_scale = s (the fold is
+ *     one fp32 multiply per weight);
+ *   - the scaled activations are those the W4A16 layer would be fed:
+ *     fl16(fl32(x) / s_j), an fp32 division rounded once to `dtype`;
+ *   - the quantized layer's output is that of the W4A16 layer: the exact
+ *     product rounded once to `dtype`; the reference W X is the exact fp64
+ *     product of the unquantized 16-bit operands;
+ *   - the norm is the Frobenius norm, and err holds its square
+ *     sum_{i,n} (Yq - Yref)^2 (same argmin);
+ *   - best is the first index of the smallest err; a NaN err is never best,
+ *     and *best = -1 when every err is NaN.
+ * Returns W4REF_EINVAL on a bad shape, or the quantizer's status.
+ */
+int w4ref_awq_search(const uint16_t *W, const uint16_t *X, int dtype, long Mc, long K, long N,
+                     long group, int sym, const float *alphas, long n_alpha, double *err,
+                     float *s_all, long *best)
+{
+    if (Mc <= 0 || K <= 0 || N <= 0 || n_alpha <= 0) return W4REF_EINVAL;
+    if (group <= 0 || group > 4096 || group % 8 != 0 || K % group != 0) return W4REF_EINVAL;
+    if (dtype != DT_F16 && dtype != DT_BF16) return W4REF_EINVAL;
+    fesetround(FE_TONEAREST);
+    const long G = K / group;
+    int status = W4REF_OK;
+    float *a = malloc(sizeof(float) * K);
+    float *wm = malloc(sizeof(float) * K);
+    float *s = malloc(sizeof(float) * K);
+    double *Yref = malloc(sizeof(double) * Mc * N);
+    double *D = malloc(sizeof(double) * Mc * N);
+    double *Xs = malloc(sizeof(double) * Mc * K);
+    double *What = malloc(sizeof(double) * N * K);
+    uint8_t *packed = malloc((size_t)N * K / 2);
+    float *scales = malloc(sizeof(float) * N * G);
+    float *zeros = malloc(sizeof(float) * N * G);
+    if (!a || !wm || !s || !Yref || !D || !Xs || !What || !packed || !scales || !zeros) {
+        status = W4REF_EINVAL;
+        goto done;
+    }
+
+    /* importance of each input channel: mean |X_ij| over the calibration rows,
+       and the weight magnitude: mean |W_nj| over the output rows */
+    for (long j = 0; j < K; ++j) {
+        double sa = 0.0, sw = 0.0;
+        for (long i = 0; i < Mc; ++i) sa += fabs(decode16(X[i * K + j], dtype));
+        for (long n = 0; n < N; ++n) sw += fabs(decode16(W[n * K + j], dtype));
+        a[j] = (float)(sa / (double)Mc);
+        wm[j] = (float)(sw / (double)N);
+    }
+
+    /* the unquantized layer's output W X on the calibration rows */
+#pragma omp parallel for schedule(static)
+    for (long i = 0; i < Mc; ++i)
+        for (long n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (long k = 0; k < K; ++k)
+                acc += decode16(X[i * K + k], dtype) * decode16(W[n * K + k], dtype);
+            Yref[i * N + n] = acc;
+        }
+
+    for (long t = 0; t < n_alpha; ++t) {
+        const double alpha = (double)alphas[t];
+        /* s_j = (a_j / w_j)^alpha */
+        for (long j = 0; j < K; ++j)
+            s[j] = (a[j] == 0.0f || wm[j] == 0.0f) ? 1.0f
+                                                   : (float)pow((double)a[j] / (double)wm[j], alpha);
+        if (s_all) memcpy(s_all + t * K, s, sizeof(float) * K);
+        /* Q(W * s): fold s into the columns, then the per-group quantizer */
+        int st = w4ref_quantize(W, dtype, K, N, group, sym, s, packed, scales, zeros);
+        if (st != W4REF_OK) {
+            status = st;
+            goto done;
+        }
+        st = w4ref_dequant(packed, scales, sym ? NULL : zeros, K, N, group, What);
+        if (st != W4REF_OK) {
+            status = st;
+            goto done;
+        }
+        /* X / s, as the 16-bit activations of the quantized layer */
+        for (long i = 0; i < Mc; ++i)
+            for (long k = 0; k < K; ++k) {
+                float x = (float)decode16(X[i * K + k], dtype);
+                Xs[i * K + k] = w4ref_round16((double)(x / s[k]), dtype);
+            }
+        /* || Q(W * s)(X / s) - W X ||^2: squared differences, then one sum in
+           (i, n) order */
+#pragma omp parallel for schedule(static)
+        for (long i = 0; i < Mc; ++i)
+            for (long n = 0; n < N; ++n) {
+                double acc = 0.0;
+                for (long k = 0; k < K; ++k) acc += Xs[i * K + k] * What[n * K + k];
+                const double d = w4ref_round16(acc, dtype) - Yref[i * N + n];
+                D[i * N + n] = d * d;
+            }
+        double e = 0.0;
+        for (long i = 0; i < Mc * N; ++i) e += D[i];
+        err[t] = e;
+    }
+
+    /* grid search: the first alpha with the smallest error */
+    *best = -1;
+    for (long t = 0; t < n_alpha; ++t)
+        if (!isnan(err[t]) && (*best < 0 || err[t] < err[*best])) *best = t;
+
+done:
+    free(a);
+    free(wm);
+    free(s);
+    free(Yref);
+    free(D);
+    free(Xs);
+    free(What);
+    free(packed);
+    free(scales);
+    free(zeros);
+    return status;
+}
