@@ -351,7 +351,7 @@ def run_ours(args, ws_, rank, local):
     sections = {}
     if rank == 0:
         want = set(args.sections.split(",")) if args.sections not in ("all", "none") else (
-            {"decode_small_m", "prefill", "quantize"} if args.sections == "all" else set())
+            {"decode_small_m", "prefill", "quantize", "awq"} if args.sections == "all" else set())
         del graphs, layer_graphs, gblock
         if "decode_small_m" in want:
             sections["decode_small_m"] = section_small_m(w4, dev, l2, pk)
@@ -359,6 +359,8 @@ def run_ours(args, ws_, rank, local):
             sections["prefill"] = section_prefill(w4, dev, pk)
         if "quantize" in want:
             sections["quantize_7b_stack"] = section_quantize(w4, dev, pk)
+        if "awq" in want:
+            sections["awq_search"] = section_awq(w4, dev, pk)
 
     cpu = None
     if rank == 0 and args.n_gpus == 1 and not args.no_cpu:
@@ -479,6 +481,57 @@ def section_quantize(w4, dev, pk):
             "bound": "hbm", "weights": nw, "ms": round(kms, 3), "gbs": round(gbs, 1),
             "frac": round(gbs / pk["hbm_gbs"], 4), "launches": len(Ws) * 4,
             "bytes_per_weight": 2 + 0.5 + 8 / GROUP}
+
+
+def awq_inputs(dev):
+    c = synth.AWQ_SEARCH
+    W = synth.weights(c["N"], c["K"], c["std"], c["seed"], outlier_frac=c["w_outlier"],
+                      dtype=c["dtype"], device=dev)
+    X = synth.activations(c["Mc"], c["K"], c["seed"], salient_frac=c["x_salient"],
+                          dtype=c["dtype"], device=dev)
+    alphas = [i / (c["n_alpha"] - 1) for i in range(c["n_alpha"])]
+    return c, W, X, alphas
+
+
+def section_awq(w4, dev, pk):
+    """One AWQ alpha search per step: 11 alphas on a 12288 x 4096 layer with
+    512 calibration rows.  Ideal time = the bytes every pass must move at the
+    measured HBM bandwidth plus the two GEMMs' flops at the measured bf16
+    tensor peak (fp16 runs at the same rate)."""
+    c, W, X, alphas = awq_inputs(dev)
+    Mc, K, N, A = c["Mc"], c["K"], c["N"], len(alphas)
+    ws = torch.empty(w4.w4_awq_search_workspace_bytes(Mc, K, N), dtype=torch.uint8, device=dev)
+    try:
+        w4.w4_awq_search(W, X, alphas, sym=c["sym"], workspace=ws)
+    except w4.W4Error as e:
+        return {"unavailable": str(e)}
+    torch.cuda.synchronize()
+    times = []
+    for r in range(8):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        w4.w4_awq_search(W, X, alphas, sym=c["sym"], workspace=ws)
+        e1.record()
+        e1.synchronize()
+        if r >= 3:
+            times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    G = K // GROUP
+    once_bytes = 2 * N * K + 2 * Mc * K + 4 * Mc * N          # statistics, Yref write
+    per_alpha_bytes = (2 * N * K + N * K / 2 + 8 * N * G      # quantize: read W, write Q
+                       + 4 * Mc * K                           # X / s
+                       + N * K / 2 + 8 * N * G + 2 * Mc * N   # layer: read Q, write Yq
+                       + 6 * Mc * N)                          # error: read Yq, Yref
+    flops = 2 * Mc * N * K * (A + 1)
+    ideal_ms = ((once_bytes + A * per_alpha_bytes) / (pk["hbm_gbs"] * 1e9)
+                + flops / (pk["bf16_tflops"] * 1e12)) * 1e3
+    return {"workload": f"AWQ alpha search, {A} alphas, Mc={Mc} calibration rows, "
+                        f"layer N={N} K={K}, asymmetric g128 fp16",
+            "bound": "hbm+tensor", "ms": round(ms, 3), "ms_per_alpha": round(ms / A, 4),
+            "alphas_per_s": round(A / (ms * 1e-3), 1), "ideal_ms": round(ideal_ms, 3),
+            "frac": round(ideal_ms / ms, 4),
+            "launches_per_search": 4 + 1 + 6 * A + 1}
 
 
 # ---------------------------------------------------------------------------- oracle arms
@@ -612,6 +665,11 @@ def run_profile_case(args):
         torch.cuda.synchronize()
         for _ in range(args.launches):
             w4.w4_quantize(W, GROUP, sym=False, col_scale=cs)
+    elif case == "awq":
+        c, W, X, alphas = awq_inputs(dev)
+        torch.cuda.synchronize()
+        for _ in range(args.launches):
+            w4.w4_awq_search(W, X, alphas, sym=c["sym"])
     else:
         raise SystemExit(f"unknown --profile case {case}")
     torch.cuda.synchronize()
@@ -627,8 +685,8 @@ def main():
     ap.add_argument("--sections", default="all")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--profile", default=None,
-                    help="decode_m1 | decode_m4..decode_m32 | prefill | quantize: run --launches "
-                         "launches of that kernel untimed (for ncu)")
+                    help="decode_m1 | decode_m4..decode_m32 | prefill | quantize | awq: run "
+                         "--launches launches of that kernel (awq: searches) untimed (for ncu)")
     ap.add_argument("--launches", type=int, default=3)
     args = ap.parse_args()
     if args.profile:

@@ -9,7 +9,9 @@
  *         scale and zero point, round, clamp, dequantize), §2.3 (per-group
  *         granularity along in_features, in_features % group == 0),
  *         §4.2 (AWQ: weights multiplied by a per-input-channel factor before
- *         quantizing).
+ *         quantizing; the factor (a/w)^alpha from mean activation and weight
+ *         magnitudes, alpha chosen by a grid search on the layer's output
+ *         error).
  *   [PTQ] "PTQ weight quantization: from GPTQ to AWQ" (jonathanding.github.io),
  *         sections "Round-to-Nearest" and "AWQ".
  *   [MF]  "Quantization method families" (inference-learning-path.pages.dev),
@@ -19,7 +21,9 @@
  *
  * Conventions shared by every entry point:
  *   - All array arguments are DEVICE pointers of the current CUDA device,
- *     allocated and owned by the caller; the library allocates no memory.
+ *     allocated and owned by the caller; the library allocates no memory
+ *     (one exception: the first w4_awq_search on a device creates a cuBLAS
+ *     handle there, which allocates cuBLAS's own workspace).
  *     Base pointers must be 16-byte aligned (else W4_ERR_UNSUPPORTED).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *     Every call only enqueues work and returns: results are ready once the
@@ -152,6 +156,60 @@ int w4a16_gemm_noalloc(const void *X, int xt, int64_t M, const uint8_t *packed,
                        void *Y, void *stream);
 
 /*
+ * w4_awq_search_workspace_bytes -- device scratch bytes w4_awq_search needs
+ * for Mc calibration rows and a K-in, N-out layer (0 for a shape it rejects).
+ * About 0.57 N K + 6 Mc N + 2 Mc K bytes, plus 8 K bytes of fp64 column
+ * partial sums per 256 rows of max(Mc, N) and the decode path's workspace
+ * when Mc <= 32.
+ */
+size_t w4_awq_search_workspace_bytes(int64_t Mc, int64_t K, int64_t N, int group);
+
+/*
+ * w4_awq_search -- AWQ per-input-channel scale search for one linear layer.
+ * [LQ] §4.2: minimise || Q(W * s)(X / s) - W X || over s_j = (a_j / w_j)^alpha,
+ * a_j = mean_i |X_ij| over the calibration rows, w_j = mean_n |W_nj|, alpha
+ * grid-searched; [PTQ] "AWQ": XW = (X diag(s)^-1)(diag(s) W).
+ *
+ *   W          [N][K] fp16 or bf16 (xt): the unquantized weight.
+ *   X          [Mc][K] same dtype: calibration activations of the layer.
+ *   group, sym the quantizer Q (w4_quantize); group must be 128.
+ *   alphas     HOST array of n_alpha (1 .. 64) values in [0, 1]; read during
+ *              the call only.
+ *   Outputs (device, caller-allocated):
+ *     err        [n_alpha] fp64: err[t] = sum_{i,n} (Yq - Yref)^2, the squared
+ *                Frobenius norm of the layer's output error at alphas[t];
+ *     best_scale [K] fp32: s at the best alpha (all ones if every err is NaN);
+ *     best_index [1] int32: the first t with the smallest err (-1 if all NaN);
+ *     packed_out, scales_out, zeros_out: nullable (all three or none); when
+ *                given, Q(W * best_scale) in the w4_quantize layout, ready for
+ *                w4a16_gemm with activations divided by best_scale.
+ *   For each alpha:
+ *     s_j  = fl32(pow(a_j / w_j, alpha)) in fp64 (s_j = 1 where a_j or w_j is 0);
+ *            a_j and w_j are fp64 sums rounded once to fp32 after the division;
+ *     Q    = w4_quantize(W, col_scale = s);
+ *     Xs   = X / s: fl32 division rounded once to the 16-bit dtype;
+ *     Yq   = w4a16_gemm(Xs, Q), the 16-bit output of the W4A16 layer;
+ *     Yref = X W^T accumulated and kept in fp32 (cuBLAS GEMM);
+ *     err  = fixed-order fp64 sum of (Yq - Yref)^2: repeated calls on the same
+ *            device give bit-identical results.
+ *   workspace / workspace_bytes: at least w4_awq_search_workspace_bytes(...)
+ *   bytes, 256-byte aligned, contents irrelevant (clobbered).  One workspace
+ *   per concurrently running search.
+ *   Returns W4_ERR_INVALID_ARG for a bad shape, count, alpha, pointer or
+ *   workspace; W4_ERR_UNSUPPORTED for group != 128, misaligned pointers or
+ *   a missing libcublas.so.12; W4_ERR_CUDA if an enqueue fails.
+ *   Besides the stream's work this call takes a process-wide lock around
+ *   its cuBLAS call; the first call on a device opens libcublas.so.12 (the
+ *   process's copy if already loaded) and creates a cuBLAS handle for that
+ *   device, kept until the process exits, so make the first call outside any
+ *   stream capture.
+ */
+int w4_awq_search(const void *W, const void *X, int xt, int64_t Mc, int64_t K, int64_t N,
+                  int group, int sym, const float *alphas, int n_alpha, double *err,
+                  float *best_scale, int *best_index, uint8_t *packed_out, float *scales_out,
+                  float *zeros_out, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * w4_device_status -- reads (and, if reset != 0, clears) the current device's
  * status word that kernels set when a bounded wait runs out.  Synchronizes the
  * device first.  Returns W4_OK, W4_ERR_TIMEOUT, or W4_ERR_CUDA if the read fails.
@@ -186,7 +244,7 @@ const char *w4_status_string(int status);
 /* ABI version of this header: (major << 16) | minor. */
 int w4_abi_version(void);
 
-#define W4A16_ABI_VERSION 0x00010000
+#define W4A16_ABI_VERSION 0x00010001
 
 #ifdef __cplusplus
 }

@@ -134,7 +134,7 @@ def awq_col_scale(Xcal: torch.Tensor) -> torch.Tensor:
     return Xcal.to(torch.float64).abs().mean(dim=0).sqrt().to(torch.float32)
 
 
-# ---- the five workloads ------------------------------------------------------------------
+# ---- the workloads ----------------------------------------------------------------------
 
 TINY = dict(name="tiny", N=256, K=512, M=1, std=0.02, seed=0, sym=True, dtype="f16")
 DECODE_M1 = dict(name="decode_m1", K=4096, Ns=(4096, 11008, 12288), M=1, std=0.02, seed=2,
@@ -149,3 +149,6 @@ STACK_7B = dict(name="quant_7b_stack", layers=32,
                         ("down", 4096, 11008)),
                 std=0.02, seed=5, sym=False, dtype="f16", w_outlier=0.001, calib_M=512,
                 x_salient=0.01)
+# AWQ alpha search on one 7B projection (qkv, 12288 x 4096) with 512 calibration rows
+AWQ_SEARCH = dict(name="awq_search", Mc=512, K=4096, N=12288, n_alpha=11, std=0.02, seed=6,
+                  sym=False, dtype="f16", w_outlier=0.001, x_salient=0.01)

@@ -45,7 +45,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert w4.w4_abi_version() == 0x00010000
+    assert w4.w4_abi_version() == 0x00010001
     assert w4.w4_status_string(0) == "W4_OK"
     assert w4.w4_status_string(1) == "W4_ERR_INVALID_ARG"
     assert w4.w4_status_string(2) == "W4_ERR_UNSUPPORTED"
@@ -128,3 +128,46 @@ def test_selftest_argument_check(lib):
     for bad in (0, 1000001):
         assert lib.w4_selftest_wait_timeout(bad, None) == w4.W4_ERR_INVALID_ARG
         assert b"timeout_us" in lib.w4_last_error()
+
+
+ALPHAS = (ctypes.c_float * 3)(0.0, 0.5, 1.0)
+BAD_ALPHAS = (ctypes.c_float * 2)(0.0, 1.5)
+E = ctypes.c_void_p(0x600000)
+F = ctypes.c_void_p(0x700000)
+WS = ctypes.c_void_p(0x10000000)
+
+
+@pytest.mark.parametrize("args,status", [
+    # (W, X, xt, Mc, K, N, group, sym, alphas, n_alpha, err, best_scale, best_index,
+    #  packed_out, scales_out, zeros_out, ws, ws_bytes)
+    ((A, B, 0, 16, 192, 64, 128, 0, ALPHAS, 3, C, D, E, None, None, None, WS, 1 << 30), 1),  # K % 128
+    ((A, B, 0, 0, 256, 64, 128, 0, ALPHAS, 3, C, D, E, None, None, None, WS, 1 << 30), 1),   # Mc 0
+    ((A, B, 0, 16, 256, 0, 128, 0, ALPHAS, 3, C, D, E, None, None, None, WS, 1 << 30), 1),   # N 0
+    ((A, B, 7, 16, 256, 64, 128, 0, ALPHAS, 3, C, D, E, None, None, None, WS, 1 << 30), 1),  # dtype
+    ((A, B, 0, 16, 256, 64, 64, 0, ALPHAS, 3, C, D, E, None, None, None, WS, 1 << 30), 2),   # group
+    ((A, B, 0, 16, 256, 64, 128, 0, ALPHAS, 0, C, D, E, None, None, None, WS, 1 << 30), 1),  # none
+    ((A, B, 0, 16, 256, 64, 128, 0, ALPHAS, 65, C, D, E, None, None, None, WS, 1 << 30), 1), # > 64
+    ((A, B, 0, 16, 256, 64, 128, 0, BAD_ALPHAS, 2, C, D, E, None, None, None, WS, 1 << 30), 1),
+    ((A, B, 0, 16, 256, 64, 128, 0, None, 3, C, D, E, None, None, None, WS, 1 << 30), 1),
+    ((None, B, 0, 16, 256, 64, 128, 0, ALPHAS, 3, C, D, E, None, None, None, WS, 1 << 30), 1),
+    ((A, B, 0, 16, 256, 64, 128, 0, ALPHAS, 3, None, D, E, None, None, None, WS, 1 << 30), 1),
+    ((A, B, 0, 16, 256, 64, 128, 0, ALPHAS, 3, C, D, None, None, None, None, WS, 1 << 30), 1),
+    ((A, B, 0, 16, 256, 64, 128, 0, ALPHAS, 3, C, D, E, F, None, None, WS, 1 << 30), 1),     # partial q
+    ((A, B, 0, 16, 256, 64, 128, 0, ALPHAS, 3, C, D, E, None, None, None, WS, 1024), 1),     # ws small
+    ((A, B, 0, 16, 256, 64, 128, 0, ALPHAS, 3, C, D, E, None, None, None,
+      ctypes.c_void_p(0x10000010), 1 << 30), 1),                                             # ws align
+    ((ctypes.c_void_p(0x100004), B, 0, 16, 256, 64, 128, 0, ALPHAS, 3, C, D, E, None, None, None,
+      WS, 1 << 30), 2),                                                                      # W align
+])
+def test_awq_search_argument_checks(lib, args, status):
+    assert lib.w4_awq_search(*args, S) == status
+
+
+def test_awq_search_workspace_size(lib):
+    Mc, K, N = 512, 4096, 12288
+    need = w4.w4_awq_search_workspace_bytes(Mc, K, N)
+    floor = N * K // 2 + 2 * N * (K // 128) * 4 + 2 * Mc * K + 2 * Mc * N + 4 * Mc * N
+    assert floor <= need <= floor + 48 * 8 * K + 64 * 1024
+    assert w4.w4_awq_search_workspace_bytes(Mc, 4000, N) == 0   # K % 128
+    assert w4.w4_awq_search_workspace_bytes(0, K, N) == 0
+    assert w4.w4_awq_search_workspace_bytes(16, K, N) >= w4.w4a16_workspace_bytes(16, K, N)

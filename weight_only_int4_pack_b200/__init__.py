@@ -12,6 +12,8 @@ pointers:
     w4_quantize(W, group=128, sym=True, col_scale=None) -> (packed, scales, zeros)
     w4a16_workspace_bytes(M, K, N, group=128) -> int
     w4a16_gemm(X, packed, scales, zeros, group=128, out=None, workspace=None) -> Y
+    w4_awq_search(W, Xcal, alphas, group=128, sym=False, quantize=False)
+        -> (err, best_scale, best_index[, (packed, scales, zeros)])
     w4_status_string(status) -> str
     w4_device_status(reset=True) -> int
 """
@@ -25,7 +27,8 @@ import torch
 __all__ = [
     "W4Error", "load", "lib_path", "w4_quantize", "w4_quantize_into", "w4a16_workspace_bytes",
     "w4a16_gemm", "w4a16_gemm_into", "w4_status_string", "w4_device_status", "w4_abi_version",
-    "w4_last_error", "w4a16_gemm_noalloc", "w4_selftest_wait_timeout",
+    "w4_last_error", "w4a16_gemm_noalloc", "w4_selftest_wait_timeout", "w4_awq_search",
+    "w4_awq_search_workspace_bytes",
     "Workspace", "W4_OK", "W4_ERR_INVALID_ARG", "W4_ERR_UNSUPPORTED", "W4_ERR_CUDA",
     "W4_ERR_TIMEOUT", "W4_F16", "W4_BF16",
 ]
@@ -75,6 +78,10 @@ def load() -> ctypes.CDLL:
     lib.w4a16_gemm_noalloc.restype = I
     lib.w4_selftest_wait_timeout.argtypes = [ctypes.c_uint, P]
     lib.w4_selftest_wait_timeout.restype = I
+    lib.w4_awq_search_workspace_bytes.argtypes = [I64, I64, I64, I]
+    lib.w4_awq_search_workspace_bytes.restype = SZ
+    lib.w4_awq_search.argtypes = [P, P, I, I64, I64, I64, I, I, P, I, P, P, P, P, P, P, P, SZ, P]
+    lib.w4_awq_search.restype = I
     lib.w4_last_error.argtypes = []
     lib.w4_last_error.restype = ctypes.c_char_p
     _lib = lib
@@ -226,3 +233,48 @@ def w4a16_gemm_noalloc(X, packed, scales, zeros=None, group: int = 128, out=None
     if st != W4_OK:
         raise W4Error("w4a16_gemm_noalloc", st)
     return Y
+
+
+def w4_awq_search_workspace_bytes(Mc: int, K: int, N: int, group: int = 128) -> int:
+    return int(load().w4_awq_search_workspace_bytes(int(Mc), int(K), int(N), int(group)))
+
+
+def w4_awq_search(W, Xcal, alphas, group: int = 128, sym: bool = False, quantize: bool = False,
+                  workspace=None, stream=None):
+    """AWQ scale search: err[t] = ||Q(W*s_t)(Xcal/s_t) - Xcal W^T||_F^2 with
+    s_t = (mean|Xcal| / mean|W|)^alphas[t] per input channel.
+
+    Returns (err fp64 [n_alpha], best_scale fp32 [K], best_index int32 [1]),
+    all on W's device, plus (packed, scales, zeros) = Q(W * best_scale) when
+    quantize=True.  `workspace` is an optional uint8 device tensor of at
+    least w4_awq_search_workspace_bytes bytes."""
+    _check_dev(W, Xcal, workspace)
+    N, K = W.shape
+    Mc = Xcal.shape[0]
+    if Xcal.dtype != W.dtype:
+        raise TypeError("W and Xcal must share one dtype")
+    a = [float(v) for v in alphas]
+    al = (ctypes.c_float * len(a))(*a)
+    lib = load()
+    need = int(lib.w4_awq_search_workspace_bytes(Mc, K, N, int(group)))
+    ws = workspace if workspace is not None else torch.empty(max(need, 256), dtype=torch.uint8,
+                                                             device=W.device)
+    dev = W.device
+    err = torch.empty(len(a), dtype=torch.float64, device=dev)
+    best_scale = torch.empty(K, dtype=torch.float32, device=dev)
+    best_index = torch.empty(1, dtype=torch.int32, device=dev)
+    q = None
+    if quantize:
+        G = K // group if group > 0 else 0
+        q = (torch.empty((N, K // 2), dtype=torch.uint8, device=dev),
+             torch.empty((N, G), dtype=torch.float32, device=dev),
+             torch.empty((N, G), dtype=torch.float32, device=dev))
+    st = lib.w4_awq_search(_p(W), _p(Xcal), _dt(W), Mc, K, N, int(group), int(bool(sym)), al,
+                           len(a), _p(err), _p(best_scale), _p(best_index),
+                           *(_p(t) for t in (q or (None, None, None))), _p(ws),
+                           ws.numel() * ws.element_size(), _stream(stream))
+    if st != W4_OK:
+        raise W4Error("w4_awq_search", st)
+    if quantize:
+        return err, best_scale, best_index, q
+    return err, best_scale, best_index
