@@ -11,7 +11,8 @@ Sources followed (see ``w4ref.c`` for the step-by-step citations):
 (zhiyuanblog.org/blog/llm-quantization) §2.2-§2.3 and §4.2, and
 "PTQ weight quantization: from GPTQ to AWQ" (jonathanding.github.io),
 sections "Round-to-Nearest" and "AWQ" (the AWQ scale search of §4.2 is
-``awq_search``).
+``awq_search``); §4.3 SmoothQuant and §4.6 FP8 for the W8A8 layer
+(``smooth_scales``, ``quant8``, ``gemm8``).
 """
 from __future__ import annotations
 
@@ -27,6 +28,8 @@ _LIB = os.path.join(_HERE, "libw4ref.so")
 
 F16 = 0
 BF16 = 1
+INT8 = 0
+E4M3 = 1
 
 OK = 0
 EINVAL = 1
@@ -71,6 +74,16 @@ def _load():
         lib.w4ref_round16.restype = ctypes.c_double
         lib.w4ref_awq_search.argtypes = [P, P, I, L, L, L, L, I, P, L, P, P, P]
         lib.w4ref_awq_search.restype = I
+        lib.w4ref_round_e4m3.argtypes = [ctypes.c_double]
+        lib.w4ref_round_e4m3.restype = ctypes.c_double
+        lib.w4ref_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+        lib.w4ref_e4m3_to_f64.restype = ctypes.c_double
+        lib.w4ref_smooth_scales.argtypes = [P, P, I, L, L, L, ctypes.c_double, P]
+        lib.w4ref_smooth_scales.restype = I
+        lib.w4ref_quant8.argtypes = [P, I, L, L, P, I, I, P, P]
+        lib.w4ref_quant8.restype = I
+        lib.w4ref_gemm8.argtypes = [P, P, I, L, L, L, ctypes.c_float, ctypes.c_float, I, P, L, P]
+        lib.w4ref_gemm8.restype = I
         lib.w4ref_threads.argtypes = []
         lib.w4ref_threads.restype = I
         lib.w4ref_set_threads.argtypes = [I]
@@ -212,3 +225,60 @@ def awq_search(W, X, dtype: int, group: int, sym: bool, alphas):
     if st != OK:
         raise OracleError(f"w4ref_awq_search status {st}")
     return err, s_all, int(best.value)
+
+
+def round_e4m3(v: float) -> float:
+    """Nearest E4M3 value to v (ties to even), saturating at +-448."""
+    return float(_load().w4ref_round_e4m3(float(v)))
+
+
+def e4m3_to_f64(c: int) -> float:
+    return float(_load().w4ref_e4m3_to_f64(int(c)))
+
+
+def smooth_scales(X, W, dtype: int, alpha: float = 0.5) -> np.ndarray:
+    """SmoothQuant factors s [K] fp32 from calibration X [Mc][K] and W [N][K]."""
+    X = _bits16(X)
+    W = _bits16(W)
+    Mc, K = X.shape
+    N = W.shape[0]
+    s = np.zeros(K, np.float32)
+    st = _load().w4ref_smooth_scales(_ptr(X), _ptr(W), dtype, Mc, K, N, float(alpha), _ptr(s))
+    if st != OK:
+        raise OracleError(f"w4ref_smooth_scales status {st}")
+    return s
+
+
+def quant8(A, dtype: int, fmt: int, col=None, col_op: int = 0):
+    """Per-tensor 8-bit quantization of A [rows][K] -> (q uint8 [rows][K], scale f32).
+    col_op: 0 none, 1 multiply by col[k], 2 divide by col[k]."""
+    A = _bits16(A)
+    rows, K = A.shape
+    if col is not None:
+        col = np.ascontiguousarray(col, dtype=np.float32)
+    q = np.zeros((rows, K), np.uint8)
+    sc = np.zeros(1, np.float32)
+    st = _load().w4ref_quant8(_ptr(A), dtype, rows, K, _ptr(col), int(col_op), int(fmt), _ptr(q),
+                              _ptr(sc))
+    if st != OK:
+        raise OracleError(f"w4ref_quant8 status {st}")
+    return q, np.float32(sc[0])
+
+
+def gemm8(Xq, Wq, fmt: int, sx, sw, dtype: int, rows=None) -> np.ndarray:
+    """W8A8 layer on quantized operands (see w4ref_gemm8): [M or len(rows)][N] fp64."""
+    Xq = np.ascontiguousarray(Xq, dtype=np.uint8)
+    Wq = np.ascontiguousarray(Wq, dtype=np.uint8)
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    if rows is not None:
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        nr = rows.shape[0]
+    else:
+        nr = M
+    Y = np.zeros((nr, N), np.float64)
+    st = _load().w4ref_gemm8(_ptr(Xq), _ptr(Wq), int(fmt), M, K, N, float(sx), float(sw), dtype,
+                             _ptr(rows), nr, _ptr(Y))
+    if st != OK:
+        raise OracleError(f"w4ref_gemm8 status {st}")
+    return Y

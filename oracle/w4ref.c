@@ -21,6 +21,9 @@
  *              before the per-group quantizer runs; s = (a/w)^alpha from the
  *              mean magnitudes of activations and weights, alpha grid-searched
  *              to minimise the layer's output error.
+ *         §4.3 SmoothQuant: s = max|X_j|^a / max|W_j|^(1-a), W*s and X/s both
+ *              quantized to INT8 per tensor (W8A8).
+ *         §4.6 FP8 E4M3: scale = max|x| / 448, cast.
  *   [PTQ] "PTQ weight quantization: from GPTQ to AWQ" (jonathanding.github.io),
  *         section "Round-to-Nearest": every weight is rounded on its own to the
  *         nearest level; section "AWQ": XW = (X diag(s)^-1)(diag(s) W).
@@ -456,4 +459,170 @@ done:
     free(scales);
     free(zeros);
     return status;
+}
+
+/* ---- W8A8: SmoothQuant factors, per-tensor INT8 / FP8 E4M3, the 8-bit GEMM -------------- */
+/*
+ *   [LQ] §4.3 SmoothQuant: s_j = max|X_j|^alpha / max|W_j|^(1-alpha) (alpha = 0.5),
+ *        clamped below at 1e-5; W' = W * s (columns), X' = X / s; both quantized
+ *        to INT8 with the symmetric formula of §2.2 (per tensor; X dynamically).
+ *   [LQ] §4.6 FP8: scale = max|x| / 448 (the largest E4M3 value), x_fp8 = cast(x / scale).
+ *   [LQ] §2.2 symmetric: s = max|x| / (2^(b-1) - 1), q = clamp(round(x / s), -qmax, qmax).
+ */
+
+#define FMT_INT8 0
+#define FMT_E4M3 1
+
+/*
+ * Nearest E4M3 value to v (ties to even) as a double: 4 significant bits,
+ * smallest normal exponent -6 (spacing 2^-9 below it), largest finite 448;
+ * magnitudes beyond 448 saturate to +-448 (no infinities in this format).
+ */
+double w4ref_round_e4m3(double v)
+{
+    if (v == 0.0 || isnan(v)) return v;
+    int e;
+    frexp(v, &e);
+    int lead = e - 1;
+    if (lead < -6) lead = -6;
+    const int q = lead - 3;
+    double r = ldexp(nearbyint(ldexp(v, -q)), q);
+    if (fabs(r) > 448.0) r = copysign(448.0, v);
+    return r;
+}
+
+/* Byte code of an E4M3 value r (exactly representable): sign, 4 exponent bits
+   (bias 7; 0 = subnormal), 3 fraction bits. */
+static uint8_t e4m3_code(double r)
+{
+    uint8_t sign = signbit(r) ? 0x80 : 0;
+    double a = fabs(r);
+    if (a == 0.0) return sign;
+    int e;
+    frexp(a, &e);
+    int lead = e - 1;
+    if (lead < -6) /* subnormal: a = f * 2^-9, f in 1..7 */
+        return sign | (uint8_t)(int)ldexp(a, 9);
+    const int frac = (int)(ldexp(a, 3 - lead)) - 8; /* a = (8 + frac) * 2^(lead-3) */
+    return sign | (uint8_t)((lead + 7) << 3) | (uint8_t)frac;
+}
+
+/* Value of an E4M3 byte (0x7F / 0xFF are NaN). */
+double w4ref_e4m3_to_f64(uint8_t c)
+{
+    const int sign = c >> 7, e = (c >> 3) & 0xF, f = c & 7;
+    double v;
+    if (e == 15 && f == 7)
+        v = NAN;
+    else if (e == 0)
+        v = ldexp((double)f, -9);
+    else
+        v = ldexp((double)(8 + f), e - 10);
+    return sign ? -v : v;
+}
+
+/*
+ * SmoothQuant factors: a_j = max_i |X_ij|, w_j = max_n |W_nj| (exact),
+ * s_j = max(fl32(fl32(a_j^alpha) / fl32(w_j^(1-alpha))), 1e-5), each power in
+ * fp64 rounded once to fp32, the quotient an fp32 division.  A channel with
+ * a_j == 0 or w_j == 0 keeps s_j = 1.
+ */
+int w4ref_smooth_scales(const uint16_t *X, const uint16_t *W, int dtype, long Mc, long K, long N,
+                        double alpha, float *s)
+{
+    if (Mc <= 0 || K <= 0 || N <= 0) return W4REF_EINVAL;
+    fesetround(FE_TONEAREST);
+    for (long j = 0; j < K; ++j) {
+        double a = 0.0, w = 0.0;
+        for (long i = 0; i < Mc; ++i) a = fmax(a, fabs(decode16(X[i * K + j], dtype)));
+        for (long n = 0; n < N; ++n) w = fmax(w, fabs(decode16(W[n * K + j], dtype)));
+        if (a == 0.0 || w == 0.0) {
+            s[j] = 1.0f;
+            continue;
+        }
+        const float num = (float)pow((double)(float)a, alpha);
+        const float den = (float)pow((double)(float)w, 1.0 - alpha);
+        float v = num / den;
+        s[j] = v < 1e-5f ? 1e-5f : v;
+    }
+    return W4REF_OK;
+}
+
+/*
+ * Per-tensor symmetric 8-bit quantization of A [rows][K] (16-bit bits).
+ * col_op: 0 none, 1 multiply column k by col[k] (the weight side, W * s),
+ * 2 divide column k by col[k] (the activation side, X / s); one fp32 op.
+ * fmt INT8: scale = fl32(amax / 127), q = clamp(rne(fl32(v / scale)), -127, 127);
+ * fmt E4M3: scale = fl32(amax / 448), q = e4m3(fl32(v / scale)).
+ * amax = 0 gives scale = 0 and every q = 0.  q is [rows][K] bytes (int8 or E4M3).
+ */
+int w4ref_quant8(const uint16_t *A, int dtype, long rows, long K, const float *col, int col_op,
+                 int fmt, uint8_t *q, float *scale_out)
+{
+    if (rows <= 0 || K <= 0 || (col_op != 0 && !col) || col_op < 0 || col_op > 2) return W4REF_EINVAL;
+    if (fmt != FMT_INT8 && fmt != FMT_E4M3) return W4REF_EINVAL;
+    fesetround(FE_TONEAREST);
+    float amax = 0.0f;
+    for (long i = 0; i < rows * K; ++i) {
+        float v = (float)decode16(A[i], dtype);
+        if (col_op == 1) v = v * col[i % K];
+        if (col_op == 2) v = v / col[i % K];
+        if (!isfinite(v)) return W4REF_ENONFINITE;
+        if (fabsf(v) > amax) amax = fabsf(v);
+    }
+    const float scale = amax / (fmt == FMT_INT8 ? 127.0f : 448.0f);
+    *scale_out = scale;
+    for (long i = 0; i < rows * K; ++i) {
+        float v = (float)decode16(A[i], dtype);
+        if (col_op == 1) v = v * col[i % K];
+        if (col_op == 2) v = v / col[i % K];
+        if (scale == 0.0f) {
+            q[i] = 0;
+            continue;
+        }
+        const float t = v / scale;
+        if (fmt == FMT_INT8)
+            q[i] = (uint8_t)(int8_t)(int)clampf(rne(t), -127.0f, 127.0f);
+        else
+            q[i] = e4m3_code(w4ref_round_e4m3((double)t));
+    }
+    return W4REF_OK;
+}
+
+/*
+ * The W8A8 layer on quantized operands: Y[m][n] from Xq [M][K] and Wq [N][K].
+ * INT8: the exact integer sum acc, then y = fl32(fl32(acc) * fl32(sx * sw))
+ *       rounded once to the 16-bit dtype (the tensor-core path's epilogue);
+ *       Y holds that 16-bit value.
+ * E4M3: Y holds the exact product sum_k x_k w_k * sx * sw in fp64 (unrounded).
+ * rows (nullable) selects the m to compute, as in w4ref_linear.
+ */
+int w4ref_gemm8(const uint8_t *Xq, const uint8_t *Wq, int fmt, long M, long K, long N, float sx,
+                float sw, int dtype, const long *rows, long nrows, double *Y)
+{
+    if (M <= 0 || K <= 0 || N <= 0) return W4REF_EINVAL;
+    if (fmt != FMT_INT8 && fmt != FMT_E4M3) return W4REF_EINVAL;
+    fesetround(FE_TONEAREST);
+    if (!rows) nrows = M;
+    const float alpha = sx * sw;
+#pragma omp parallel for schedule(static)
+    for (long r = 0; r < nrows; ++r) {
+        const long m = rows ? rows[r] : r;
+        if (m < 0 || m >= M) continue;
+        for (long n = 0; n < N; ++n) {
+            if (fmt == FMT_INT8) {
+                long long acc = 0;
+                for (long k = 0; k < K; ++k)
+                    acc += (long long)(int8_t)Xq[m * K + k] * (long long)(int8_t)Wq[n * K + k];
+                const float y = (float)acc * alpha;
+                Y[r * N + n] = w4ref_round16((double)y, dtype);
+            } else {
+                double acc = 0.0;
+                for (long k = 0; k < K; ++k)
+                    acc += w4ref_e4m3_to_f64(Xq[m * K + k]) * w4ref_e4m3_to_f64(Wq[n * K + k]);
+                Y[r * N + n] = acc * (double)sx * (double)sw;
+            }
+        }
+    }
+    return W4REF_OK;
 }
