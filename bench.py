@@ -351,7 +351,8 @@ def run_ours(args, ws_, rank, local):
     sections = {}
     if rank == 0:
         want = set(args.sections.split(",")) if args.sections not in ("all", "none") else (
-            {"decode_small_m", "prefill", "quantize", "awq"} if args.sections == "all" else set())
+            {"decode_small_m", "prefill", "quantize", "awq", "w8a8"} if args.sections == "all"
+            else set())
         del graphs, layer_graphs, gblock
         if "decode_small_m" in want:
             sections["decode_small_m"] = section_small_m(w4, dev, l2, pk)
@@ -361,6 +362,8 @@ def run_ours(args, ws_, rank, local):
             sections["quantize_7b_stack"] = section_quantize(w4, dev, pk)
         if "awq" in want:
             sections["awq_search"] = section_awq(w4, dev, pk)
+        if "w8a8" in want:
+            sections["w8a8"] = section_w8a8(w4, dev, pk)
 
     cpu = None
     if rank == 0 and args.n_gpus == 1 and not args.no_cpu:
@@ -534,6 +537,68 @@ def section_awq(w4, dev, pk):
             "launches_per_search": 4 + 1 + 6 * A + 1}
 
 
+def w8a8_inputs(w4, dev, fmt):
+    c = synth.W8A8
+    X = synth.activations(c["M"], c["K"], c["seed"], salient_frac=c["x_salient"],
+                          dtype=c["dtype"], device=dev)
+    W = synth.weights(c["N"], c["K"], c["std"], c["seed"], dtype=c["dtype"], device=dev)
+    s = w4.w8_smooth_scales(X, W, c["alpha"]) if fmt == w4.W8_INT8 else None
+    wq, sw = w4.w8_quantize(W, fmt, s, w4.W8_COL_MUL if s is not None else w4.W8_COL_NONE)
+    xq, sx = w4.w8_quantize(X, fmt, s, w4.W8_COL_DIV if s is not None else w4.W8_COL_NONE)
+    return c, X, s, wq, sw, xq, sx
+
+
+def section_w8a8(w4, dev, pk):
+    """The W8A8 layer at M = 2048, K = 4096, N = 11008 (bf16 in and out):
+    SmoothQuant INT8 and FP8 E4M3.  `gemm` times the 8-bit tcgen05 GEMM alone
+    on quantized operands, `linear` the layer with the on-the-fly activation
+    quantization; L2 is flushed between launches.  The 8-bit dense peak is the
+    measured bf16 peak x 2 (the nominal int8 / fp8 : bf16 ratio)."""
+    peak8 = 2 * pk["bf16_tflops"]
+    out = {"workload": "W8A8 M=2048 K=4096 N=11008 bf16, per-tensor scales "
+                       "(INT8 with SmoothQuant alpha=0.5; FP8 E4M3)",
+           "bound": "tensor", "peak_tops": peak8,
+           "peak_note": "measured bf16 burst x 2 (nominal 8-bit : bf16 ratio)"}
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+    for name, fmt in (("int8", w4.W8_INT8), ("fp8_e4m3", w4.W8_E4M3)):
+        try:
+            c, X, s, wq, sw, xq, sx = w8a8_inputs(w4, dev, fmt)
+            M, K, N = c["M"], c["K"], c["N"]
+            Y = torch.empty((M, N), dtype=X.dtype, device=dev)
+            ws = torch.empty(w4.w8a8_workspace_bytes(M, K), dtype=torch.uint8, device=dev)
+            w4.w8_gemm(xq, sx, wq, sw, fmt, X.dtype, out=Y)
+            w4.w8a8_linear(X, wq, sw, fmt, s=s, out=Y, workspace=ws)
+        except w4.W4Error as e:
+            out[name] = {"unavailable": str(e)}
+            continue
+        torch.cuda.synchronize()
+        res = {}
+        for part, fn in (("gemm", lambda: w4.w8_gemm(xq, sx, wq, sw, fmt, X.dtype, out=Y)),
+                         ("linear", lambda: w4.w8a8_linear(X, wq, sw, fmt, s=s, out=Y,
+                                                           workspace=ws))):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn()
+            times = []
+            for r in range(23):
+                flush.zero_()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                g.replay()
+                e1.record()
+                e1.synchronize()
+                if r >= 3:
+                    times.append(e0.elapsed_time(e1))
+            kms = statistics.median(times)
+            tops = 2 * M * N * K / (kms * 1e-3) / 1e12
+            res[part] = {"us": round(kms * 1e3, 1), "tops": round(tops, 1),
+                         "frac": round(tops / peak8, 4)}
+            del g
+        out[name] = res
+    return out
+
+
 # ---------------------------------------------------------------------------- oracle arms
 
 def oracle_step(layer_sets_host, Xbits, dtype):
@@ -665,6 +730,12 @@ def run_profile_case(args):
         torch.cuda.synchronize()
         for _ in range(args.launches):
             w4.w4_quantize(W, GROUP, sym=False, col_scale=cs)
+    elif case in ("w8a8_int8", "w8a8_fp8"):
+        fmt = w4.W8_INT8 if case.endswith("int8") else w4.W8_E4M3
+        c, X, s, wq, sw, xq, sx = w8a8_inputs(w4, dev, fmt)
+        torch.cuda.synchronize()
+        for _ in range(args.launches):
+            w4.w8_gemm(xq, sx, wq, sw, fmt, X.dtype)
     elif case == "awq":
         c, W, X, alphas = awq_inputs(dev)
         torch.cuda.synchronize()
@@ -685,7 +756,8 @@ def main():
     ap.add_argument("--sections", default="all")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--profile", default=None,
-                    help="decode_m1 | decode_m4..decode_m32 | prefill | quantize | awq: run "
+                    help="decode_m1 | decode_m4..decode_m32 | prefill | quantize | awq | w8a8_int8 | "
+                         "w8a8_fp8: run "
                          "--launches launches of that kernel (awq: searches) untimed (for ncu)")
     ap.add_argument("--launches", type=int, default=3)
     args = ap.parse_args()

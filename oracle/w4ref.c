@@ -605,6 +605,8 @@ int w4ref_gemm8(const uint8_t *Xq, const uint8_t *Wq, int fmt, long M, long K, l
     fesetround(FE_TONEAREST);
     if (!rows) nrows = M;
     const float alpha = sx * sw;
+    double e4m3[256]; /* value of every E4M3 byte, from the decoder above */
+    for (int c = 0; c < 256; ++c) e4m3[c] = w4ref_e4m3_to_f64((uint8_t)c);
 #pragma omp parallel for schedule(static)
     for (long r = 0; r < nrows; ++r) {
         const long m = rows ? rows[r] : r;
@@ -619,7 +621,7 @@ int w4ref_gemm8(const uint8_t *Xq, const uint8_t *Wq, int fmt, long M, long K, l
             } else {
                 double acc = 0.0;
                 for (long k = 0; k < K; ++k)
-                    acc += w4ref_e4m3_to_f64(Xq[m * K + k]) * w4ref_e4m3_to_f64(Wq[n * K + k]);
+                    acc += e4m3[Xq[m * K + k]] * e4m3[Wq[n * K + k]];
                 Y[r * N + n] = acc * (double)sx * (double)sw;
             }
         }

@@ -152,3 +152,6 @@ STACK_7B = dict(name="quant_7b_stack", layers=32,
 # AWQ alpha search on one 7B projection (qkv, 12288 x 4096) with 512 calibration rows
 AWQ_SEARCH = dict(name="awq_search", Mc=512, K=4096, N=12288, n_alpha=11, std=0.02, seed=6,
                   sym=False, dtype="f16", w_outlier=0.001, x_salient=0.01)
+# W8A8 layer (SmoothQuant INT8 / FP8 E4M3) on the prefill shape
+W8A8 = dict(name="w8a8", M=2048, K=4096, N=11008, std=0.02, seed=7, dtype="bf16",
+            x_salient=0.01, alpha=0.5)

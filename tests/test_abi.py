@@ -171,3 +171,54 @@ def test_awq_search_workspace_size(lib):
     assert w4.w4_awq_search_workspace_bytes(Mc, 4000, N) == 0   # K % 128
     assert w4.w4_awq_search_workspace_bytes(0, K, N) == 0
     assert w4.w4_awq_search_workspace_bytes(16, K, N) >= w4.w4a16_workspace_bytes(16, K, N)
+
+
+@pytest.mark.parametrize("args,status", [
+    # (A, at, rows, K, col, col_op, fmt, q, scale)
+    ((A, 0, 4, 40, None, 0, 0, B, C), 1),      # K % 16
+    ((A, 0, 0, 64, None, 0, 0, B, C), 1),      # rows 0
+    ((A, 3, 4, 64, None, 0, 0, B, C), 1),      # dtype
+    ((A, 0, 4, 64, None, 0, 2, B, C), 1),      # fmt
+    ((A, 0, 4, 64, None, 3, 0, B, C), 1),      # col_op
+    ((A, 0, 4, 64, None, 1, 0, B, C), 1),      # col missing for W8_COL_MUL
+    ((None, 0, 4, 64, None, 0, 0, B, C), 1),
+    ((A, 0, 4, 64, None, 0, 0, None, C), 1),
+    ((A, 0, 4, 64, None, 0, 0, B, None), 1),
+    ((ctypes.c_void_p(0x100008), 0, 4, 64, None, 0, 0, B, C), 2),  # misaligned A
+    ((A, 0, 4, 64, None, 0, 0, B, ctypes.c_void_p(0x300004)), 2),  # misaligned scale
+])
+def test_w8_quantize_argument_checks(lib, args, status):
+    assert lib.w8_quantize(*args, S) == status
+
+
+@pytest.mark.parametrize("args,status", [
+    # (Xq, x_scale, Wq, w_scale, fmt, M, K, N, Y, yt)
+    ((A, B, C, D, 0, 4, 40, 8, E, 0), 1),      # K % 16
+    ((A, B, C, D, 0, 0, 64, 8, E, 0), 1),      # M 0
+    ((A, B, C, D, 0, 4, 64, 0, E, 0), 1),      # N 0
+    ((A, B, C, D, 5, 4, 64, 8, E, 0), 1),      # fmt
+    ((A, B, C, D, 0, 4, 64, 8, E, 9), 1),      # out dtype
+    ((A, B, C, D, 0, 4, 140000, 8, E, 0), 2),  # INT8 accumulator range
+    ((A, None, C, D, 0, 4, 64, 8, E, 0), 1),
+    ((A, B, C, D, 0, 4, 64, 8, None, 0), 1),
+    ((A, B, ctypes.c_void_p(0x300008), D, 0, 4, 64, 8, E, 0), 2),
+])
+def test_w8_gemm_argument_checks(lib, args, status):
+    assert lib.w8_gemm(*args, S) == status
+
+
+def test_w8_smooth_and_linear_argument_checks(lib):
+    F = ctypes.c_float
+    # (X, W, xt, Mc, K, N, alpha, s, ws, ws_bytes)
+    assert lib.w8_smooth_scales(A, B, 0, 8, 64, 16, F(1.5), C, WS, 8 * 64, S) == 1
+    assert lib.w8_smooth_scales(A, B, 0, 8, 64, 16, F(0.5), C, WS, 8 * 63, S) == 1
+    assert lib.w8_smooth_scales(A, B, 0, 8, 40, 16, F(0.5), C, WS, 8 * 64, S) == 1
+    assert lib.w8_smooth_scales(A, B, 0, 0, 64, 16, F(0.5), C, WS, 8 * 64, S) == 1
+    assert lib.w8_smooth_scales(A, None, 0, 8, 64, 16, F(0.5), C, WS, 8 * 64, S) == 1
+    assert w4.w8a8_workspace_bytes(3, 64) == 512
+    assert w4.w8a8_workspace_bytes(3, 40) == 0
+    # (X, xt, M, K, s, fmt, Wq, w_scale, N, Y, ws, ws_bytes)
+    assert lib.w8a8_linear(A, 0, 3, 64, None, 0, B, C, 8, D, WS, 256, S) == 1   # small ws
+    assert lib.w8a8_linear(A, 0, 3, 64, None, 0, B, C, 8, D,
+                           ctypes.c_void_p(0x10000010), 512, S) == 2            # ws align
+    assert lib.w8a8_linear(A, 0, 3, 64, None, 0, B, C, 0, D, WS, 512, S) == 1   # N 0

@@ -14,6 +14,10 @@ pointers:
     w4a16_gemm(X, packed, scales, zeros, group=128, out=None, workspace=None) -> Y
     w4_awq_search(W, Xcal, alphas, group=128, sym=False, quantize=False)
         -> (err, best_scale, best_index[, (packed, scales, zeros)])
+    w8_smooth_scales(X, W, alpha=0.5) -> s
+    w8_quantize(A, fmt, col=None, col_op=W8_COL_NONE) -> (q, scale)
+    w8_gemm(Xq, x_scale, Wq, w_scale, fmt, dtype) -> Y
+    w8a8_linear(X, Wq, w_scale, fmt, s=None) -> Y
     w4_status_string(status) -> str
     w4_device_status(reset=True) -> int
 """
@@ -28,13 +32,17 @@ __all__ = [
     "W4Error", "load", "lib_path", "w4_quantize", "w4_quantize_into", "w4a16_workspace_bytes",
     "w4a16_gemm", "w4a16_gemm_into", "w4_status_string", "w4_device_status", "w4_abi_version",
     "w4_last_error", "w4a16_gemm_noalloc", "w4_selftest_wait_timeout", "w4_awq_search",
-    "w4_awq_search_workspace_bytes",
+    "w4_awq_search_workspace_bytes", "w8_smooth_scales", "w8_quantize", "w8_gemm",
+    "w8a8_workspace_bytes", "w8a8_linear", "W8_INT8", "W8_E4M3", "W8_COL_NONE", "W8_COL_MUL",
+    "W8_COL_DIV",
     "Workspace", "W4_OK", "W4_ERR_INVALID_ARG", "W4_ERR_UNSUPPORTED", "W4_ERR_CUDA",
     "W4_ERR_TIMEOUT", "W4_F16", "W4_BF16",
 ]
 
 W4_OK, W4_ERR_INVALID_ARG, W4_ERR_UNSUPPORTED, W4_ERR_CUDA, W4_ERR_TIMEOUT = 0, 1, 2, 3, 4
 W4_F16, W4_BF16 = 0, 1
+W8_INT8, W8_E4M3 = 0, 1
+W8_COL_NONE, W8_COL_MUL, W8_COL_DIV = 0, 1, 2
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(_PKG, "lib", "libw4a16.so")
@@ -82,6 +90,17 @@ def load() -> ctypes.CDLL:
     lib.w4_awq_search_workspace_bytes.restype = SZ
     lib.w4_awq_search.argtypes = [P, P, I, I64, I64, I64, I, I, P, I, P, P, P, P, P, P, P, SZ, P]
     lib.w4_awq_search.restype = I
+    F = ctypes.c_float
+    lib.w8_smooth_scales.argtypes = [P, P, I, I64, I64, I64, F, P, P, SZ, P]
+    lib.w8_smooth_scales.restype = I
+    lib.w8_quantize.argtypes = [P, I, I64, I64, P, I, I, P, P, P]
+    lib.w8_quantize.restype = I
+    lib.w8_gemm.argtypes = [P, P, P, P, I, I64, I64, I64, P, I, P]
+    lib.w8_gemm.restype = I
+    lib.w8a8_workspace_bytes.argtypes = [I64, I64]
+    lib.w8a8_workspace_bytes.restype = SZ
+    lib.w8a8_linear.argtypes = [P, I, I64, I64, P, I, P, P, I64, P, P, SZ, P]
+    lib.w8a8_linear.restype = I
     lib.w4_last_error.argtypes = []
     lib.w4_last_error.restype = ctypes.c_char_p
     _lib = lib
@@ -278,3 +297,67 @@ def w4_awq_search(W, Xcal, alphas, group: int = 128, sym: bool = False, quantize
     if quantize:
         return err, best_scale, best_index, q
     return err, best_scale, best_index
+
+
+# ---- W8A8 (SmoothQuant INT8 / FP8 E4M3) ---------------------------------------------------
+
+def w8_smooth_scales(X, W, alpha: float = 0.5, stream=None):
+    """SmoothQuant factors s [K] fp32 from calibration X [Mc][K] and W [N][K]."""
+    _check_dev(X, W)
+    Mc, K = X.shape
+    N = W.shape[0]
+    s = torch.empty(K, dtype=torch.float32, device=X.device)
+    ws = torch.empty(8 * K, dtype=torch.uint8, device=X.device)
+    st = load().w8_smooth_scales(_p(X), _p(W), _dt(X), Mc, K, N, float(alpha), _p(s), _p(ws),
+                                 ws.numel(), _stream(stream))
+    if st != W4_OK:
+        raise W4Error("w8_smooth_scales", st)
+    return s
+
+
+def w8_quantize(A, fmt: int, col=None, col_op: int = W8_COL_NONE, stream=None):
+    """Per-tensor 8-bit quantization of A [rows][K] -> (q uint8 [rows][K], scale f32 [2]
+    holding (scale, amax))."""
+    _check_dev(A, col)
+    rows, K = A.shape
+    q = torch.empty((rows, K), dtype=torch.uint8, device=A.device)
+    scale = torch.empty(2, dtype=torch.float32, device=A.device)
+    st = load().w8_quantize(_p(A), _dt(A), rows, K, _p(col), int(col_op), int(fmt), _p(q),
+                            _p(scale), _stream(stream))
+    if st != W4_OK:
+        raise W4Error("w8_quantize", st)
+    return q, scale
+
+
+def w8_gemm(Xq, x_scale, Wq, w_scale, fmt: int, dtype=torch.float16, out=None, stream=None):
+    """Y [M][N] = (Xq Wq^T) * x_scale[0] * w_scale[0] on 8-bit operands."""
+    _check_dev(Xq, x_scale, Wq, w_scale, out)
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    Y = out if out is not None else torch.empty((M, N), dtype=dtype, device=Xq.device)
+    st = load().w8_gemm(_p(Xq), _p(x_scale), _p(Wq), _p(w_scale), int(fmt), M, K, N, _p(Y),
+                        _dt(Y), _stream(stream))
+    if st != W4_OK:
+        raise W4Error("w8_gemm", st)
+    return Y
+
+
+def w8a8_workspace_bytes(M: int, K: int) -> int:
+    return int(load().w8a8_workspace_bytes(int(M), int(K)))
+
+
+def w8a8_linear(X, Wq, w_scale, fmt: int, s=None, out=None, workspace=None, stream=None):
+    """The W8A8 layer: X [M][K] (16-bit) divided by s, quantized per tensor on
+    the fly, times the quantized weights Wq [N][K]; Y [M][N] in X's dtype."""
+    _check_dev(X, Wq, w_scale, s, out, workspace)
+    M, K = X.shape
+    N = Wq.shape[0]
+    Y = out if out is not None else torch.empty((M, N), dtype=X.dtype, device=X.device)
+    need = w8a8_workspace_bytes(M, K)
+    ws = workspace if workspace is not None else torch.empty(max(need, 256), dtype=torch.uint8,
+                                                             device=X.device)
+    st = load().w8a8_linear(_p(X), _dt(X), M, K, _p(s), int(fmt), _p(Wq), _p(w_scale), N, _p(Y),
+                            _p(ws), ws.numel() * ws.element_size(), _stream(stream))
+    if st != W4_OK:
+        raise W4Error("w8a8_linear", st)
+    return Y
