@@ -84,6 +84,10 @@ def _load():
         lib.w4ref_quant8.restype = I
         lib.w4ref_gemm8.argtypes = [P, P, I, L, L, L, ctypes.c_float, ctypes.c_float, I, P, L, P]
         lib.w4ref_gemm8.restype = I
+        lib.w4ref_gptq_quantize.argtypes = [P, I, L, L, L, I, P, P, P, P]
+        lib.w4ref_gptq_quantize.restype = I
+        lib.w4ref_gptq_hessian.argtypes = [P, I, L, L, P]
+        lib.w4ref_gptq_hessian.restype = I
         lib.w4ref_threads.argtypes = []
         lib.w4ref_threads.restype = I
         lib.w4ref_set_threads.argtypes = [I]
@@ -282,3 +286,52 @@ def gemm8(Xq, Wq, fmt: int, sx, sw, dtype: int, rows=None) -> np.ndarray:
     if st != OK:
         raise OracleError(f"w4ref_gemm8 status {st}")
     return Y
+
+
+def gptq_hessian(X, dtype: int) -> np.ndarray:
+    """H = 2 X^T X in fp64 ([K][K]) from calibration activations X [Mc][K]."""
+    X = _bits16(X)
+    Mc, K = X.shape
+    H = np.zeros((K, K), np.float64)
+    st = _load().w4ref_gptq_hessian(_ptr(X), dtype, Mc, K, _ptr(H))
+    if st != OK:
+        raise OracleError(f"w4ref_gptq_hessian status {st}")
+    return H
+
+
+def gptq_inverse_factor(H: np.ndarray, percdamp: float = 0.01) -> np.ndarray:
+    """U (upper, fp64) with U^T U = (H + lambda I)^-1, lambda = percdamp * mean(diag H).
+
+    Library steps (numpy.linalg): the inverse of the damped Hessian, then its
+    Cholesky factor; U = L^T for the lower factor L."""
+    H = np.array(H, dtype=np.float64, copy=True)
+    lam = percdamp * float(np.mean(np.diag(H)))
+    H[np.diag_indices_from(H)] += lam
+    Hinv = np.linalg.inv(H)
+    Hinv = (Hinv + Hinv.T) / 2
+    return np.linalg.cholesky(Hinv).T.copy()
+
+
+def gptq_quantize(W, dtype: int, U, group: int, sym: bool):
+    """The GPTQ column loop over W [N][K] given the fp32 factor U [K][K];
+    returns (packed, scales, zeros) in the w4_quantize layout."""
+    W = _bits16(W)
+    N, K = W.shape
+    U = np.ascontiguousarray(U, dtype=np.float32)
+    assert U.shape == (K, K)
+    G = K // group
+    packed = np.zeros((N, K // 2), np.uint8)
+    scales = np.zeros((N, G), np.float32)
+    zeros = np.zeros((N, G), np.float32)
+    st = _load().w4ref_gptq_quantize(_ptr(W), dtype, K, N, group, int(bool(sym)), _ptr(U),
+                                     _ptr(packed), _ptr(scales), _ptr(zeros))
+    if st != OK:
+        raise OracleError(f"w4ref_gptq_quantize status {st}")
+    return packed, scales, zeros
+
+
+def gptq(W, X, dtype: int, group: int, sym: bool, percdamp: float = 0.01):
+    """Whole GPTQ for one layer: Hessian, damped inverse factor (rounded to
+    fp32), column loop.  Returns (packed, scales, zeros, U32)."""
+    U32 = gptq_inverse_factor(gptq_hessian(X, dtype), percdamp).astype(np.float32)
+    return (*gptq_quantize(W, dtype, U32, group, sym), U32)

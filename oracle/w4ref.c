@@ -628,3 +628,129 @@ int w4ref_gemm8(const uint8_t *Xq, const uint8_t *Wq, int fmt, long M, long K, l
     }
     return W4REF_OK;
 }
+
+
+/* ---- GPTQ: Hessian-guided column-by-column quantization ------------------------------- */
+/*
+ *   [LQ] §4.1 GPTQ: minimise ||WX - W^X||_F^2 with H = 2 X X^T; quantize one
+ *        column at a time and push each column's error onto the columns not yet
+ *        quantized through the inverse Hessian (delta_j = (w_j - q_j) / [H^-1]_jj,
+ *        W[:, j+1:] -= delta_j H^-1[j, j+1:]); in practice through a Cholesky
+ *        factor of H^-1, with the updates to later blocks batched.
+ *   [PTQ] section "GPTQ": lazy batch updates every 128 columns.
+ *   Here X is [Mc][K] (rows = calibration samples), so H = 2 X^T X is [K][K].
+ *   U is the upper Cholesky factor of H^-1 (H^-1 = U^T U); its row j gives
+ *   [H_F^-1]_jj and the update row of the still-unquantized set F at step j.
+ */
+
+/* Group parameters (the RTN quantizer's formulas above) of w[0..g-1]. */
+static void group_params(const float *w, long g, int sym, float *s_out, float *z_out)
+{
+    if (sym) {
+        float amax = 0.0f;
+        for (long i = 0; i < g; ++i)
+            if (fabsf(w[i]) > amax) amax = fabsf(w[i]);
+        *s_out = amax / 7.0f;
+        *z_out = 8.0f;
+    } else {
+        float mn = w[0], mx = w[0];
+        for (long i = 1; i < g; ++i) {
+            if (w[i] < mn) mn = w[i];
+            if (w[i] > mx) mx = w[i];
+        }
+        const float s = (mx - mn) / 15.0f;
+        *s_out = s;
+        *z_out = s == 0.0f ? 0.0f : clampf(rne((-mn) / s), 0.0f, 15.0f) + 0.0f;
+    }
+}
+
+/* Stored code u of w under (s, z): the RTN quantizer's rounding and clamp. */
+static int code_of(float w, float s, float z, int sym)
+{
+    if (s == 0.0f) return (int)z;
+    if (sym) return (int)clampf(rne(w / s), -7.0f, 7.0f) + 8;
+    return (int)clampf(rne(w / s + z), 0.0f, 15.0f);
+}
+
+/*
+ * The GPTQ column loop for W [N][K] (16-bit bits) given U [K][K] fp32
+ * (row-major; only the upper triangle k >= j is read).  block == group:
+ * each group's parameters are taken from the row's current weights when the
+ * loop reaches the group (all earlier blocks' updates applied, none of its
+ * own).  Every update is fp32:
+ *   in the block, after column j:  w_k = fma(-err_j, U[j][k], w_k), k > j;
+ *   err_j = (w_j - (u_j - z) * s) / U[j][j];
+ *   after the block, for each later k: acc = fma chain over the block's j in
+ *   order (acc = fma(err_j, U[j][k], acc) from 0), then w_k = w_k - acc.
+ * Outputs in the w4_quantize layout: packed [N][K/2], scales and zeros [N][K/group].
+ */
+int w4ref_gptq_quantize(const uint16_t *W, int dtype, long K, long N, long group, int sym,
+                        const float *U, uint8_t *packed, float *scales, float *zeros)
+{
+    if (K <= 0 || N <= 0 || group <= 0 || group > 4096 || group % 8 != 0 || K % group != 0)
+        return W4REF_EINVAL;
+    fesetround(FE_TONEAREST);
+    const long G = K / group;
+    int status = W4REF_OK;
+#pragma omp parallel
+    {
+        float *w = malloc(sizeof(float) * K);
+        float *err = malloc(sizeof(float) * group);
+        uint8_t *u = malloc(K);
+        if (!w || !err || !u) {
+#pragma omp atomic write
+            status = W4REF_EINVAL;
+        }
+#pragma omp for schedule(static)
+        for (long n = 0; n < N; ++n) {
+            if (!w || !err || !u) continue;
+            for (long k = 0; k < K; ++k) w[k] = (float)decode16(W[n * K + k], dtype);
+            for (long g = 0; g < G; ++g) {
+                const long b0 = g * group;
+                float s, z;
+                group_params(w + b0, group, sym, &s, &z);
+                scales[n * G + g] = s;
+                zeros[n * G + g] = z;
+                for (long jj = 0; jj < group; ++jj) {
+                    const long j = b0 + jj;
+                    const int c = code_of(w[j], s, z, sym);
+                    u[j] = (uint8_t)c;
+                    const float deq = (float)c - z;
+                    const float e = (w[j] - deq * s) / U[j * K + j];
+                    err[jj] = e;
+                    for (long k = j + 1; k < b0 + group; ++k) w[k] = fmaf(-e, U[j * K + k], w[k]);
+                }
+                for (long k = b0 + group; k < K; ++k) {
+                    float acc = 0.0f;
+                    for (long jj = 0; jj < group; ++jj) acc = fmaf(err[jj], U[(b0 + jj) * K + k], acc);
+                    w[k] = w[k] - acc;
+                }
+            }
+            for (long j8 = 0; j8 < K / 8; ++j8) {
+                uint32_t word = 0;
+                for (int i = 0; i < 8; ++i) word |= (uint32_t)(u[j8 * 8 + SIGMA[i]] & 0xF) << (4 * i);
+                uint8_t *dst = packed + n * (K / 2) + j8 * 4;
+                for (int b = 0; b < 4; ++b) dst[b] = (uint8_t)(word >> (8 * b));
+            }
+        }
+        free(w);
+        free(err);
+        free(u);
+    }
+    return status;
+}
+
+/* H = 2 X^T X in fp64 ([K][K]) from X [Mc][K] (16-bit bits). */
+int w4ref_gptq_hessian(const uint16_t *X, int dtype, long Mc, long K, double *H)
+{
+    if (Mc <= 0 || K <= 0) return W4REF_EINVAL;
+#pragma omp parallel for schedule(static)
+    for (long a = 0; a < K; ++a)
+        for (long b = 0; b < K; ++b) {
+            double acc = 0.0;
+            for (long i = 0; i < Mc; ++i)
+                acc += decode16(X[i * K + a], dtype) * decode16(X[i * K + b], dtype);
+            H[a * K + b] = 2.0 * acc;
+        }
+    return W4REF_OK;
+}
