@@ -351,7 +351,8 @@ def run_ours(args, ws_, rank, local):
     sections = {}
     if rank == 0:
         want = set(args.sections.split(",")) if args.sections not in ("all", "none") else (
-            {"decode_small_m", "prefill", "quantize", "awq", "w8a8"} if args.sections == "all"
+            {"decode_small_m", "prefill", "quantize", "awq", "w8a8", "gptq"}
+            if args.sections == "all"
             else set())
         del graphs, layer_graphs, gblock
         if "decode_small_m" in want:
@@ -364,6 +365,8 @@ def run_ours(args, ws_, rank, local):
             sections["awq_search"] = section_awq(w4, dev, pk)
         if "w8a8" in want:
             sections["w8a8"] = section_w8a8(w4, dev, pk)
+        if "gptq" in want:
+            sections["gptq"] = section_gptq(w4, dev, pk)
 
     cpu = None
     if rank == 0 and args.n_gpus == 1 and not args.no_cpu:
@@ -599,6 +602,61 @@ def section_w8a8(w4, dev, pk):
     return out
 
 
+def gptq_inputs(dev):
+    c = synth.GPTQ
+    W = synth.weights(c["N"], c["K"], c["std"], c["seed"], outlier_frac=c["w_outlier"],
+                      dtype=c["dtype"], device=dev)
+    X = synth.activations(c["Mc"], c["K"], c["seed"], salient_frac=c["x_salient"],
+                          dtype=c["dtype"], device=dev)
+    return c, W, X
+
+
+def section_gptq(w4, dev, pk):
+    """GPTQ of the qkv projection of a 7B layer (12288 x 4096) with 512
+    calibration rows.  `whole` = w4_gptq (Hessian, damping, factorization --
+    which synchronizes once -- and the column loop); `column_loop` =
+    w4_gptq_quantize alone.  The loop is bound by the fp32 FMAs of its lazy
+    updates, N * 128^2 * G (G - 1) / 2 for G = K / 128 blocks, against the
+    fp32 FMA peak from the unit counts: 148 SMs x 128 lanes x 2 flops x the
+    maximum SM clock (1965 MHz)."""
+    c, W, X = gptq_inputs(dev)
+    N, K, Mc = c["N"], c["K"], c["Mc"]
+    ws = torch.empty(w4.w4_gptq_workspace_bytes(Mc, K, N), dtype=torch.uint8, device=dev)
+    try:
+        p, s, z, U = w4.w4_gptq(W, X, sym=c["sym"], percdamp=c["percdamp"], return_u=True,
+                                workspace=ws)
+    except w4.W4Error as e:
+        return {"unavailable": str(e)}
+    torch.cuda.synchronize()
+    res = {}
+    for part, fn in (("whole", lambda: w4.w4_gptq(W, X, sym=c["sym"], percdamp=c["percdamp"],
+                                                  workspace=ws)),
+                     ("column_loop", lambda: w4.w4_gptq_quantize(W, U, sym=c["sym"],
+                                                                 workspace=ws))):
+        times = []
+        for r in range(6):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            if r >= 1:
+                times.append(e0.elapsed_time(e1))
+        res[part] = {"ms": round(statistics.median(times), 3)}
+    G = K // GROUP
+    lazy_flops = 2.0 * N * GROUP * GROUP * G * (G - 1) / 2
+    peak = 148 * 128 * 2 * 1965e6 / 1e12  # clocks.max.sm of the B200: 1965 MHz
+    tf = lazy_flops / (res["column_loop"]["ms"] * 1e-3) / 1e12
+    return {"workload": f"GPTQ N={N} K={K}, {Mc} calibration rows, asymmetric g128 fp16, "
+                        f"percdamp {c['percdamp']}",
+            "bound": "alu", "whole_ms": res["whole"]["ms"],
+            "column_loop_ms": res["column_loop"]["ms"],
+            "lazy_update_tflops": round(tf, 2), "peak_fp32_tflops": round(peak, 1),
+            "frac": round(tf / peak, 4),
+            "peak_note": "fp32 FMA lanes x max clock (148 x 128 x 2 x 1965 MHz)"}
+
+
 # ---------------------------------------------------------------------------- oracle arms
 
 def oracle_step(layer_sets_host, Xbits, dtype):
@@ -736,6 +794,11 @@ def run_profile_case(args):
         torch.cuda.synchronize()
         for _ in range(args.launches):
             w4.w8_gemm(xq, sx, wq, sw, fmt, X.dtype)
+    elif case == "gptq":
+        c, W, X = gptq_inputs(dev)
+        torch.cuda.synchronize()
+        for _ in range(args.launches):
+            w4.w4_gptq(W, X, sym=c["sym"], percdamp=c["percdamp"])
     elif case == "awq":
         c, W, X, alphas = awq_inputs(dev)
         torch.cuda.synchronize()
@@ -756,7 +819,7 @@ def main():
     ap.add_argument("--sections", default="all")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--profile", default=None,
-                    help="decode_m1 | decode_m4..decode_m32 | prefill | quantize | awq | w8a8_int8 | "
+                    help="decode_m1 | decode_m4..decode_m32 | prefill | quantize | awq | gptq | w8a8_int8 | "
                          "w8a8_fp8: run "
                          "--launches launches of that kernel (awq: searches) untimed (for ncu)")
     ap.add_argument("--launches", type=int, default=3)

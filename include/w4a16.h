@@ -8,6 +8,8 @@
  *         parameter), §2.2 (symmetric and asymmetric integer quantization,
  *         scale and zero point, round, clamp, dequantize), §2.3 (per-group
  *         granularity along in_features, in_features % group == 0),
+ *         §4.1 (GPTQ: H = 2XX^T, column-wise quantization with the error
+ *         pushed through the inverse Hessian),
  *         §4.2 (AWQ: weights multiplied by a per-input-channel factor before
  *         quantizing; the factor (a/w)^alpha from mean activation and weight
  *         magnitudes, alpha chosen by a grid search on the layer's output
@@ -22,8 +24,8 @@
  * Conventions shared by every entry point:
  *   - All array arguments are DEVICE pointers of the current CUDA device,
  *     allocated and owned by the caller; the library allocates no memory
- *     (one exception: the first w4_awq_search on a device creates a cuBLAS
- *     handle there, which allocates cuBLAS's own workspace).
+ *     (exceptions: the first w4_awq_search or w4_gptq on a device creates
+ *     cuBLAS / cuSOLVER handles there, which allocate their own workspace).
  *     Base pointers must be 16-byte aligned (else W4_ERR_UNSUPPORTED).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *     Every call only enqueues work and returns: results are ready once the
@@ -210,6 +212,58 @@ int w4_awq_search(const void *W, const void *X, int xt, int64_t Mc, int64_t K, i
                   float *zeros_out, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * w4_gptq_workspace_bytes / w4_gptq_quantize_workspace_bytes -- device
+ * scratch bytes of w4_gptq and w4_gptq_quantize (0 for a shape they reject):
+ * about 4 K^2 + 4 N K + 512 N bytes (w4_gptq) and 4 N K + 512 N (the loop).
+ */
+size_t w4_gptq_workspace_bytes(int64_t Mc, int64_t K, int64_t N, int group);
+size_t w4_gptq_quantize_workspace_bytes(int64_t K, int64_t N, int group);
+
+/*
+ * w4_gptq -- GPTQ quantization of one layer ([LQ] §4.1; [PTQ] "GPTQ"):
+ * minimise ||W X^T - W^ X^T|| column by column, pushing each column's
+ * rounding error onto the columns not yet quantized through the inverse
+ * Hessian, with lazy updates every 128 columns.
+ *
+ *   W          [N][K] fp16 or bf16 (xt), the weight; X [Mc][K] the same dtype,
+ *              the layer's calibration activations.
+ *   group      must be 128 (the GPTQ block); K % 128 == 0; sym as w4_quantize.
+ *   percdamp   damping in [0, 1]: H = 2 X^T X + percdamp * mean(diag) * I
+ *              (the usual 0.01; the pages give none).
+ *   Outputs: packed / scales / zeros in the w4_quantize layout (w4a16_gemm
+ *   consumes them unchanged); U_out nullable [K][K] fp32: the factor used
+ *   (row-major, upper triangle; the strictly lower part is unspecified).
+ *   Steps: H in fp32 (cuBLAS GEMM, fp32 accumulation); U = the upper
+ *   Cholesky factor of H^-1 (cuSOLVER potrf, potri, potrf in fp32); then the
+ *   column loop of w4_gptq_quantize.  The call synchronizes `stream` once,
+ *   after the factorization, to read its status: W4_ERR_INVALID_ARG if the
+ *   damped Hessian is not positive definite (e.g. X all zero with damping).
+ *   The first call on a device opens libcublas.so.12 and libcusolver.so.11
+ *   and creates their handles (kept until exit); a missing library returns
+ *   W4_ERR_UNSUPPORTED.
+ *   workspace: w4_gptq_workspace_bytes bytes, 256-byte aligned, clobbered.
+ */
+int w4_gptq(const void *W, const void *X, int xt, int64_t Mc, int64_t K, int64_t N, int group,
+            int sym, float percdamp, uint8_t *packed, float *scales, float *zeros, float *U_out,
+            void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * w4_gptq_quantize -- the GPTQ column loop alone, given U.
+ *   W [N][K] (wt), U [K][K] fp32 row-major, upper triangle read (U^T U is the
+ *   damped inverse Hessian; U[j][j] > 0).  For every row, for each block of
+ *   128 columns: the group's scale and zero point from the row's current
+ *   weights (w4_quantize's formulas, fp32); then for each column j in order:
+ *   code u_j (w4_quantize's rounding), err_j = (w_j - (u_j - z) s) / U[j][j],
+ *   w_k = fma(-err_j, U[j][k], w_k) for the block's k > j; after the block,
+ *   for every later column k: w_k = w_k - acc with acc the fp32 fma chain of
+ *   err_j U[j][k] over the block's j in order.  All fp32, IEEE division, so
+ *   the codes are a fixed function of W and U.  Asynchronous; no library.
+ */
+int w4_gptq_quantize(const void *W, int wt, int64_t K, int64_t N, int group, int sym,
+                     const float *U, uint8_t *packed, float *scales, float *zeros,
+                     void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * w4_device_status -- reads (and, if reset != 0, clears) the current device's
  * status word that kernels set when a bounded wait runs out.  Synchronizes the
  * device first.  Returns W4_OK, W4_ERR_TIMEOUT, or W4_ERR_CUDA if the read fails.
@@ -244,7 +298,7 @@ const char *w4_status_string(int status);
 /* ABI version of this header: (major << 16) | minor. */
 int w4_abi_version(void);
 
-#define W4A16_ABI_VERSION 0x00010001
+#define W4A16_ABI_VERSION 0x00010002
 
 #ifdef __cplusplus
 }

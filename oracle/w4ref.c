@@ -744,13 +744,17 @@ int w4ref_gptq_quantize(const uint16_t *W, int dtype, long K, long N, long group
 int w4ref_gptq_hessian(const uint16_t *X, int dtype, long Mc, long K, double *H)
 {
     if (Mc <= 0 || K <= 0) return W4REF_EINVAL;
+    double *Xt = malloc(sizeof(double) * Mc * K); /* X transposed, decoded: Xt[a][i] */
+    if (!Xt) return W4REF_EINVAL;
+    for (long i = 0; i < Mc; ++i)
+        for (long a = 0; a < K; ++a) Xt[a * Mc + i] = decode16(X[i * K + a], dtype);
 #pragma omp parallel for schedule(static)
     for (long a = 0; a < K; ++a)
         for (long b = 0; b < K; ++b) {
             double acc = 0.0;
-            for (long i = 0; i < Mc; ++i)
-                acc += decode16(X[i * K + a], dtype) * decode16(X[i * K + b], dtype);
+            for (long i = 0; i < Mc; ++i) acc += Xt[a * Mc + i] * Xt[b * Mc + i];
             H[a * K + b] = 2.0 * acc;
         }
+    free(Xt);
     return W4REF_OK;
 }

@@ -155,3 +155,6 @@ AWQ_SEARCH = dict(name="awq_search", Mc=512, K=4096, N=12288, n_alpha=11, std=0.
 # W8A8 layer (SmoothQuant INT8 / FP8 E4M3) on the prefill shape
 W8A8 = dict(name="w8a8", M=2048, K=4096, N=11008, std=0.02, seed=7, dtype="bf16",
             x_salient=0.01, alpha=0.5)
+# GPTQ on one 7B projection (qkv, 12288 x 4096) with 512 calibration rows
+GPTQ = dict(name="gptq", N=12288, K=4096, Mc=512, std=0.02, seed=8, dtype="f16", sym=False,
+            w_outlier=0.001, x_salient=0.01, percdamp=0.01)

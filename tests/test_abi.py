@@ -45,7 +45,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert w4.w4_abi_version() == 0x00010001
+    assert w4.w4_abi_version() == 0x00010002
     assert w4.w4_status_string(0) == "W4_OK"
     assert w4.w4_status_string(1) == "W4_ERR_INVALID_ARG"
     assert w4.w4_status_string(2) == "W4_ERR_UNSUPPORTED"
@@ -222,3 +222,35 @@ def test_w8_smooth_and_linear_argument_checks(lib):
     assert lib.w8a8_linear(A, 0, 3, 64, None, 0, B, C, 8, D,
                            ctypes.c_void_p(0x10000010), 512, S) == 2            # ws align
     assert lib.w8a8_linear(A, 0, 3, 64, None, 0, B, C, 0, D, WS, 512, S) == 1   # N 0
+
+
+def test_gptq_argument_checks(lib):
+    F = ctypes.c_float
+    # (W, X, xt, Mc, K, N, group, sym, percdamp, packed, scales, zeros, U_out, ws, ws_bytes)
+    ok = (A, B, 0, 64, 256, 32, 128, 0, F(0.01), C, D, E, None, WS, 1 << 30)
+    def call(**kw):
+        a = list(ok)
+        names = ["W", "X", "xt", "Mc", "K", "N", "group", "sym", "pd", "p", "s", "z", "U", "ws",
+                 "wsb"]
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return lib.w4_gptq(*a, S)
+    assert call(K=192) == 1            # K % 128
+    assert call(group=64) == 2         # group must be 128
+    assert call(Mc=0) == 1
+    assert call(N=0) == 1
+    assert call(xt=4) == 1
+    assert call(pd=F(-0.5)) == 1
+    assert call(W=None) == 1
+    assert call(wsb=1024) == 1
+    assert call(ws=ctypes.c_void_p(0x10000010)) == 1
+    assert call(X=ctypes.c_void_p(0x200008)) == 2
+    need = w4.w4_gptq_workspace_bytes(64, 256, 32)
+    assert need >= 4 * 256 * 256 + 4 * 32 * 256
+    assert w4.w4_gptq_workspace_bytes(64, 200, 32) == 0
+    q = w4.w4_gptq_quantize_workspace_bytes(256, 32)
+    assert 4 * 32 * 256 + 512 * 32 <= q < need
+    # (W, wt, K, N, group, sym, U, packed, scales, zeros, ws, ws_bytes)
+    assert lib.w4_gptq_quantize(A, 0, 256, 32, 128, 0, None, C, D, E, WS, q, S) == 1
+    assert lib.w4_gptq_quantize(A, 0, 256, 32, 128, 0, B, C, D, E, WS, q - 1, S) == 1
+    assert lib.w4_gptq_quantize(A, 0, 256, 32, 32, 0, B, C, D, E, WS, q, S) == 2

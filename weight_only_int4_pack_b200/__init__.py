@@ -14,6 +14,8 @@ pointers:
     w4a16_gemm(X, packed, scales, zeros, group=128, out=None, workspace=None) -> Y
     w4_awq_search(W, Xcal, alphas, group=128, sym=False, quantize=False)
         -> (err, best_scale, best_index[, (packed, scales, zeros)])
+    w4_gptq(W, Xcal, group=128, sym=False, percdamp=0.01) -> (packed, scales, zeros[, U])
+    w4_gptq_quantize(W, U, group=128, sym=False) -> (packed, scales, zeros)
     w8_smooth_scales(X, W, alpha=0.5) -> s
     w8_quantize(A, fmt, col=None, col_op=W8_COL_NONE) -> (q, scale)
     w8_gemm(Xq, x_scale, Wq, w_scale, fmt, dtype) -> Y
@@ -32,7 +34,8 @@ __all__ = [
     "W4Error", "load", "lib_path", "w4_quantize", "w4_quantize_into", "w4a16_workspace_bytes",
     "w4a16_gemm", "w4a16_gemm_into", "w4_status_string", "w4_device_status", "w4_abi_version",
     "w4_last_error", "w4a16_gemm_noalloc", "w4_selftest_wait_timeout", "w4_awq_search",
-    "w4_awq_search_workspace_bytes", "w8_smooth_scales", "w8_quantize", "w8_gemm",
+    "w4_awq_search_workspace_bytes", "w4_gptq", "w4_gptq_quantize", "w4_gptq_workspace_bytes",
+    "w4_gptq_quantize_workspace_bytes", "w8_smooth_scales", "w8_quantize", "w8_gemm",
     "w8a8_workspace_bytes", "w8a8_linear", "W8_INT8", "W8_E4M3", "W8_COL_NONE", "W8_COL_MUL",
     "W8_COL_DIV",
     "Workspace", "W4_OK", "W4_ERR_INVALID_ARG", "W4_ERR_UNSUPPORTED", "W4_ERR_CUDA",
@@ -91,6 +94,14 @@ def load() -> ctypes.CDLL:
     lib.w4_awq_search.argtypes = [P, P, I, I64, I64, I64, I, I, P, I, P, P, P, P, P, P, P, SZ, P]
     lib.w4_awq_search.restype = I
     F = ctypes.c_float
+    lib.w4_gptq_workspace_bytes.argtypes = [I64, I64, I64, I]
+    lib.w4_gptq_workspace_bytes.restype = SZ
+    lib.w4_gptq_quantize_workspace_bytes.argtypes = [I64, I64, I]
+    lib.w4_gptq_quantize_workspace_bytes.restype = SZ
+    lib.w4_gptq.argtypes = [P, P, I, I64, I64, I64, I, I, F, P, P, P, P, P, SZ, P]
+    lib.w4_gptq.restype = I
+    lib.w4_gptq_quantize.argtypes = [P, I, I64, I64, I, I, P, P, P, P, P, SZ, P]
+    lib.w4_gptq_quantize.restype = I
     lib.w8_smooth_scales.argtypes = [P, P, I, I64, I64, I64, F, P, P, SZ, P]
     lib.w8_smooth_scales.restype = I
     lib.w8_quantize.argtypes = [P, I, I64, I64, P, I, I, P, P, P]
@@ -297,6 +308,62 @@ def w4_awq_search(W, Xcal, alphas, group: int = 128, sym: bool = False, quantize
     if quantize:
         return err, best_scale, best_index, q
     return err, best_scale, best_index
+
+
+# ---- GPTQ ------------------------------------------------------------------------------------
+
+def w4_gptq_workspace_bytes(Mc: int, K: int, N: int, group: int = 128) -> int:
+    return int(load().w4_gptq_workspace_bytes(int(Mc), int(K), int(N), int(group)))
+
+
+def w4_gptq_quantize_workspace_bytes(K: int, N: int, group: int = 128) -> int:
+    return int(load().w4_gptq_quantize_workspace_bytes(int(K), int(N), int(group)))
+
+
+def _q_out(N, K, group, dev):
+    G = K // group if group > 0 else 0
+    return (torch.empty((N, K // 2), dtype=torch.uint8, device=dev),
+            torch.empty((N, G), dtype=torch.float32, device=dev),
+            torch.empty((N, G), dtype=torch.float32, device=dev))
+
+
+def w4_gptq(W, Xcal, group: int = 128, sym: bool = False, percdamp: float = 0.01,
+            return_u: bool = False, workspace=None, stream=None):
+    """GPTQ of W [N][K] with calibration activations Xcal [Mc][K] ->
+    (packed, scales, zeros) in the w4_quantize layout (+ U [K][K] fp32 when
+    return_u).  Synchronizes the stream once (factorization status)."""
+    _check_dev(W, Xcal, workspace)
+    N, K = W.shape
+    Mc = Xcal.shape[0]
+    if Xcal.dtype != W.dtype:
+        raise TypeError("W and Xcal must share one dtype")
+    p, s, z = _q_out(N, K, group, W.device)
+    U = torch.empty((K, K), dtype=torch.float32, device=W.device) if return_u else None
+    need = w4_gptq_workspace_bytes(Mc, K, N, group)
+    ws = workspace if workspace is not None else torch.empty(max(need, 256), dtype=torch.uint8,
+                                                             device=W.device)
+    st = load().w4_gptq(_p(W), _p(Xcal), _dt(W), Mc, K, N, int(group), int(bool(sym)),
+                        float(percdamp), _p(p), _p(s), _p(z), _p(U), _p(ws),
+                        ws.numel() * ws.element_size(), _stream(stream))
+    if st != W4_OK:
+        raise W4Error("w4_gptq", st)
+    return (p, s, z, U) if return_u else (p, s, z)
+
+
+def w4_gptq_quantize(W, U, group: int = 128, sym: bool = False, workspace=None, stream=None):
+    """The GPTQ column loop over W [N][K] given the fp32 factor U [K][K]."""
+    _check_dev(W, U, workspace)
+    N, K = W.shape
+    p, s, z = _q_out(N, K, group, W.device)
+    need = w4_gptq_quantize_workspace_bytes(K, N, group)
+    ws = workspace if workspace is not None else torch.empty(max(need, 256), dtype=torch.uint8,
+                                                             device=W.device)
+    st = load().w4_gptq_quantize(_p(W), _dt(W), K, N, int(group), int(bool(sym)), _p(U), _p(p),
+                                 _p(s), _p(z), _p(ws), ws.numel() * ws.element_size(),
+                                 _stream(stream))
+    if st != W4_OK:
+        raise W4Error("w4_gptq_quantize", st)
+    return p, s, z
 
 
 # ---- W8A8 (SmoothQuant INT8 / FP8 E4M3) ---------------------------------------------------

@@ -13,8 +13,8 @@
 //   1. column statistics (colabs_partial + colabs_finish): fp64 partial sums
 //      of |.| over chunks of kChunkRows rows, summed in chunk order, divided
 //      by the row count in fp64 and rounded once to fp32;
-//   2. the unquantized layer's output Yref = X W^T in fp32 (cuBLAS, fp32
-//      accumulation; a plain dense GEMM, done once per call);
+//   2. the unquantized layer's output Yref = X W^T in fp32 (cuBLAS through
+//      w4_libs.cu, fp32 accumulation; a plain dense GEMM, done once per call);
 //   3. per alpha: s (awq_scale); Q(W * s) with the library's quantizer
 //      (col_scale = s); X / s rounded to the 16-bit dtype (scale_activations);
 //      Yq = the W4A16 layer (decode path for Mc <= 32, tcgen05 path above);
@@ -27,13 +27,10 @@
 // quantizer reads W (100 MB) and writes the codes (25 MB), the layer reads the
 // codes and X / s, and the error pass reads Yq (12.6 MB) and Yref (25 MB).
 
-#include <cublas_v2.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
-#include <dlfcn.h>
 
 #include <math.h>
-#include <mutex>
 
 #include "w4_half.cuh"
 #include "w4_internal.cuh"
@@ -213,76 +210,15 @@ __global__ void __launch_bounds__(256) awq_select(const double *__restrict__ err
         best_scale[c] = b < 0 ? 1.0f : channel_scale(a[c], w[c], alpha);
 }
 
-// ---- cuBLAS, loaded on first use ------------------------------------------------------
-//
-// The library does not link cuBLAS: the search is the only user of it, and
-// the GEMM entry points must load where cuBLAS is absent.  The first search
-// on a device opens libcublas.so.12 (the process's copy when one is already
-// loaded, e.g. by PyTorch) and creates one handle per device, kept for the
-// life of the process.
-
-using PFN_create = cublasStatus_t (*)(cublasHandle_t *);
-using PFN_set_stream = cublasStatus_t (*)(cublasHandle_t, cudaStream_t);
-using PFN_gemm_ex = cublasStatus_t (*)(cublasHandle_t, cublasOperation_t, cublasOperation_t, int,
-                                       int, int, const void *, const void *, cudaDataType, int,
-                                       const void *, cudaDataType, int, const void *, void *,
-                                       cudaDataType, int, cublasComputeType_t, cublasGemmAlgo_t);
-
-constexpr int kMaxDevices = 64;
-std::mutex g_blas_mu;
-PFN_create g_create = nullptr;
-PFN_set_stream g_set_stream = nullptr;
-PFN_gemm_ex g_gemm_ex = nullptr;
-cublasHandle_t g_handle[kMaxDevices] = {};
-
-int blas_handle(cublasHandle_t *out) {
-    const char *fn = "w4_awq_search";
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
-    if (dev < 0 || dev >= kMaxDevices) return set_error(W4_ERR_CUDA, fn, "device ordinal out of range");
-    if (!g_gemm_ex) {
-        void *h = dlopen("libcublas.so.12", RTLD_NOW | RTLD_LOCAL);
-        if (!h) return set_error(W4_ERR_UNSUPPORTED, fn, "libcublas.so.12 could not be loaded");
-        g_create = reinterpret_cast<PFN_create>(dlsym(h, "cublasCreate_v2"));
-        g_set_stream = reinterpret_cast<PFN_set_stream>(dlsym(h, "cublasSetStream_v2"));
-        g_gemm_ex = reinterpret_cast<PFN_gemm_ex>(dlsym(h, "cublasGemmEx"));
-        if (!g_create || !g_set_stream || !g_gemm_ex) {
-            g_gemm_ex = nullptr;
-            return set_error(W4_ERR_UNSUPPORTED, fn, "libcublas.so.12 lacks cublasGemmEx");
-        }
-    }
-    if (!g_handle[dev]) {
-        cublasHandle_t h = nullptr;
-        if (g_create(&h) != CUBLAS_STATUS_SUCCESS)
-            return set_error(W4_ERR_CUDA, fn, "cublasCreate failed");
-        g_handle[dev] = h;
-    }
-    *out = g_handle[dev];
-    return W4_OK;
-}
-
-// Yref [Mc][N] fp32 = X [Mc][K] * W [N][K]^T.  Column-major view: Yref^T
-// (N x Mc, ld N) = W^T-view (op T of the K x N matrix W, ld K) * X^T-view
-// (the K x Mc matrix X, ld K).
+// Yref [Mc][N] fp32 = X [Mc][K] * W [N][K]^T (cuBLAS).  Column-major view:
+// Yref^T (N x Mc, ld N) = op T of the K x N matrix W (ld K) times the K x Mc
+// matrix X (ld K).
 int reference_gemm(const void *W, const void *X, int xt, int64_t Mc, int64_t K, int64_t N,
                    float *Yref, cudaStream_t stream) {
-    std::lock_guard<std::mutex> lk(g_blas_mu);
-    cublasHandle_t h = nullptr;
-    int st = blas_handle(&h);
-    if (st != W4_OK) return st;
-    if (g_set_stream(h, stream) != CUBLAS_STATUS_SUCCESS)
-        return set_error(W4_ERR_CUDA, "w4_awq_search", "cublasSetStream failed");
-    const float one = 1.0f, zero = 0.0f;
-    const cudaDataType dt = xt == W4_F16 ? CUDA_R_16F : CUDA_R_16BF;
-    const cublasStatus_t bs =
-        g_gemm_ex(h, CUBLAS_OP_T, CUBLAS_OP_N, static_cast<int>(N), static_cast<int>(Mc),
-                  static_cast<int>(K), &one, W, dt, static_cast<int>(K), X, dt,
-                  static_cast<int>(K), &zero, Yref, CUDA_R_32F, static_cast<int>(N),
-                  CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
-    if (bs != CUBLAS_STATUS_SUCCESS)
-        return set_error(W4_ERR_CUDA, "w4_awq_search", "cublasGemmEx (reference output) failed");
-    return W4_OK;
+    return blas_gemm_f32("w4_awq_search (reference output)", true, false, static_cast<int>(N),
+                         static_cast<int>(Mc), static_cast<int>(K), 1.0f, W, xt,
+                         static_cast<int>(K), X, xt, static_cast<int>(K), 0.0f, Yref,
+                         static_cast<int>(N), stream);
 }
 
 // ---- workspace layout -------------------------------------------------------------------

@@ -1,0 +1,399 @@
+// w4_gptq.cu -- GPTQ: per-group INT4 quantization that pushes each column's
+// rounding error onto the columns not yet quantized through the inverse
+// Hessian of the layer's calibration activations.
+//
+// Method: "LLM quantization methods: principles and implementation"
+// (zhiyuanblog.org/blog/llm-quantization) §4.1: minimise ||WX - W^X||_F^2,
+// H = 2 X X^T, quantize column by column, delta_j = (w_j - q_j) / [H^-1]_jj,
+// W[:, j+1:] -= delta_j H^-1[j, j+1:], with a Cholesky factor of H^-1 in
+// practice; "PTQ weight quantization: from GPTQ to AWQ", section "GPTQ":
+// lazy batch updates every 128 columns.  Here the calibration rows are the
+// rows of X [Mc][K], so H = 2 X^T X is [K][K].
+//
+// One call of w4_gptq, on the caller's stream:
+//   1. H = 2 X^T X in fp32 (cuBLAS GEMM, fp32 accumulation);
+//   2. damping: H_jj += percdamp * mean(diag H) (one CTA, fixed-order sum);
+//   3. U = upper Cholesky factor of H^-1 (cuSOLVER potrf, potri, potrf);
+//      the stream is synchronized once here to read the factorization status;
+//   4. the column loop (also alone as w4_gptq_quantize, given U):
+//      gptq_widen: Wf = fp32 copy of W;
+//      per 128-column block b (block = group):
+//        gptq_block: one warp per weight row, lane l holding columns
+//          4l..4l+3 of the block: the group's scale / zero point from the
+//          row's current weights (the RTN quantizer's formulas), then for
+//          each column j in order: code, err_j = (w_j - (u_j - z) s) / U_jj,
+//          w_k = fma(-err_j, U_jk, w_k) for the block's k > j; writes the
+//          packed codes, scale, zero point and err[n][0..127];
+//        gptq_lazy: Wf[:, later k] -= err[:, block] U[block, later k], each
+//          element as one fp32 fma chain over the block's 128 columns in
+//          order followed by one subtraction (a SIMT tile GEMM whose
+//          per-element order is fixed, so the result is reproducible bit for
+//          bit; 128 x 128 output tiles, 8 x 8 per thread).
+// Rows are independent given U: every decision of row n depends only on W[n]
+// and U, so the parallelism is over rows (block step) and over rows x later
+// columns (lazy update).  Outputs use the w4_quantize layout, so w4a16_gemm
+// consumes them unchanged.
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "w4_half.cuh"
+#include "w4_internal.cuh"
+
+namespace w4 {
+namespace {
+
+constexpr int kBlock = 128;  // GPTQ block = quantization group
+constexpr int kLT = 128;     // lazy update: output tile rows and columns
+constexpr int kLJ = 16;      // lazy update: block columns per shared-memory stage
+
+__global__ void __launch_bounds__(256) gptq_widen(const uint16_t *__restrict__ W, int wt,
+                                                  int64_t n8, float *__restrict__ Wf) {
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(W) + i);
+        float f[8];
+        if (wt == W4_F16)
+            widen8<W4_F16>(v, f);
+        else
+            widen8<W4_BF16>(v, f);
+        reinterpret_cast<float4 *>(Wf)[2 * i] = make_float4(f[0], f[1], f[2], f[3]);
+        reinterpret_cast<float4 *>(Wf)[2 * i + 1] = make_float4(f[4], f[5], f[6], f[7]);
+    }
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ float warp_min(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// Stored code of w under (s, z): sym  u = clamp(rne(w / s), -7, 7) + 8;
+// asym u = clamp(rne(fl(w / s) + z), 0, 15); a zero scale gives u = z.
+template <int SYM>
+__device__ __forceinline__ int code_of(float w, float s, float z) {
+    if (s == 0.0f) return static_cast<int>(z);
+    if (SYM) return static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(w, s)), -7.0f), 7.0f)) + 8;
+    return static_cast<int>(fminf(fmaxf(rintf(__fadd_rn(__fdiv_rn(w, s), z)), 0.0f), 15.0f));
+}
+
+// One warp per weight row n; block b0 .. b0 + 127 of the row.
+template <int SYM>
+__global__ void __launch_bounds__(256) gptq_block(float *__restrict__ Wf, const float *__restrict__ U,
+                                                  int64_t N, int64_t K, int64_t b0,
+                                                  uint8_t *__restrict__ packed,
+                                                  float *__restrict__ scales,
+                                                  float *__restrict__ zeros,
+                                                  float *__restrict__ Err) {
+    const int lane = threadIdx.x & 31;
+    const int64_t n = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    if (n >= N) return;  // warp-uniform
+    const int64_t G = K / kBlock;
+    float *wrow = Wf + n * K + b0;
+    const float4 wv = *reinterpret_cast<const float4 *>(wrow + 4 * lane);
+    float w[4] = {wv.x, wv.y, wv.z, wv.w};
+
+    // the group's parameters from the current weights
+    float s, z;
+    if (SYM) {
+        const float amax = warp_max(fmaxf(fmaxf(fabsf(w[0]), fabsf(w[1])), fmaxf(fabsf(w[2]), fabsf(w[3]))));
+        s = __fdiv_rn(amax, 7.0f);
+        z = 8.0f;
+    } else {
+        const float mn = warp_min(fminf(fminf(w[0], w[1]), fminf(w[2], w[3])));
+        const float mx = warp_max(fmaxf(fmaxf(w[0], w[1]), fmaxf(w[2], w[3])));
+        s = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+        z = s == 0.0f ? 0.0f
+                      : __fadd_rn(fminf(fmaxf(rintf(__fdiv_rn(-mn, s)), 0.0f), 15.0f), 0.0f);
+    }
+
+    const float *ublk = U + b0 * K + b0;  // U[b0 + j][b0 + k] = ublk[j * K + k]
+    int my_code[4] = {0, 0, 0, 0};
+    float my_err[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll 1
+    for (int jj = 0; jj < 32; ++jj) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int j = 4 * jj + i;
+            const float wj = __shfl_sync(0xffffffffu, w[i], jj);
+            const int c = code_of<SYM>(wj, s, z);
+            const float deq = __fmul_rn(__fsub_rn(static_cast<float>(c), z), s);
+            const float e = __fdiv_rn(__fsub_rn(wj, deq), __ldg(ublk + static_cast<int64_t>(j) * K + j));
+            if (lane == jj) {
+                my_code[i] = c;
+                my_err[i] = e;
+            }
+            // columns k = 4 lane + i2 > j of the block
+            if (4 * lane + 3 > j) {
+                const float4 u4 = __ldg(reinterpret_cast<const float4 *>(ublk + static_cast<int64_t>(j) * K + 4 * lane));
+                const float uk[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+                for (int i2 = 0; i2 < 4; ++i2)
+                    if (4 * lane + i2 > j) w[i2] = __fmaf_rn(-e, uk[i2], w[i2]);
+            }
+        }
+    }
+
+    // codes: lanes 2m and 2m + 1 hold k = 8m..8m+3 and 8m+4..8m+7 of word m;
+    // nibble i of the word holds k = 8m + {0,2,4,6,1,3,5,7}[i]
+    const uint32_t mine = my_code[0] | (my_code[1] << 4) | (my_code[2] << 8) | (my_code[3] << 12);
+    const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
+    if ((lane & 1) == 0) {
+        const uint32_t c0 = mine & 15, c1 = (mine >> 4) & 15, c2 = (mine >> 8) & 15, c3 = (mine >> 12) & 15;
+        const uint32_t t0 = other & 15, t1 = (other >> 4) & 15, t2 = (other >> 8) & 15, t3 = (other >> 12) & 15;
+        const uint32_t word = c0 | (c2 << 4) | (t0 << 8) | (t2 << 12) | (c1 << 16) | (c3 << 20) |
+                              (t1 << 24) | (t3 << 28);
+        reinterpret_cast<uint32_t *>(packed + n * (K / 2) + b0 / 2)[lane / 2] = word;
+    }
+    reinterpret_cast<float4 *>(Err + n * kBlock)[lane] =
+        make_float4(my_err[0], my_err[1], my_err[2], my_err[3]);
+    if (lane == 0) {
+        scales[n * G + b0 / kBlock] = s;
+        zeros[n * G + b0 / kBlock] = z;
+    }
+}
+
+// Wf[n][k] -= sum_{j < 128} Err[n][j] * U[b0 + j][k] for k >= b0 + 128: per
+// element acc = fma(Err[n][j], U[b0+j][k], acc) for j = 0, 1, ..., 127 from
+// acc = 0, then Wf = Wf - acc.  Tile 128 rows x 128 columns, 256 threads,
+// thread (ty, tx) owns rows {4ty..4ty+3, 64+4ty..64+4ty+3} and the same
+// pattern of columns.
+__global__ void __launch_bounds__(256) gptq_lazy(float *__restrict__ Wf, const float *__restrict__ Err,
+                                                 const float *__restrict__ U, int64_t N, int64_t K,
+                                                 int64_t b0) {
+    __shared__ __align__(16) float Es[kLJ][kLT];
+    __shared__ __align__(16) float Us[kLJ][kLT];
+    const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
+    const int64_t n0 = static_cast<int64_t>(blockIdx.y) * kLT;
+    const int64_t k0 = b0 + kBlock + static_cast<int64_t>(blockIdx.x) * kLT;
+    float acc[8][8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[r][c] = 0.0f;
+
+    for (int j0 = 0; j0 < kBlock; j0 += kLJ) {
+        {   // Es[jj][r] = Err[n0 + r][j0 + jj]: thread t loads row t / 2, 8 columns
+            const int r = t >> 1, h = (t & 1) * 8;
+            float4 e0 = make_float4(0.f, 0.f, 0.f, 0.f), e1 = e0;
+            if (n0 + r < N) {
+                const float4 *src = reinterpret_cast<const float4 *>(Err + (n0 + r) * kBlock + j0 + h);
+                e0 = src[0];
+                e1 = src[1];
+            }
+            Es[h + 0][r] = e0.x; Es[h + 1][r] = e0.y; Es[h + 2][r] = e0.z; Es[h + 3][r] = e0.w;
+            Es[h + 4][r] = e1.x; Es[h + 5][r] = e1.y; Es[h + 6][r] = e1.z; Es[h + 7][r] = e1.w;
+        }
+        {   // Us[jj][c] = U[b0 + j0 + jj][k0 + c]: thread t loads row t / 16, 8 columns
+            const int jj = t >> 4, c = (t & 15) * 8;
+            const float4 *src = reinterpret_cast<const float4 *>(U + (b0 + j0 + jj) * K + k0 + c);
+            *reinterpret_cast<float4 *>(&Us[jj][c]) = src[0];
+            *reinterpret_cast<float4 *>(&Us[jj][c + 4]) = src[1];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int jj = 0; jj < kLJ; ++jj) {
+            const float4 a0 = *reinterpret_cast<const float4 *>(&Es[jj][4 * ty]);
+            const float4 a1 = *reinterpret_cast<const float4 *>(&Es[jj][64 + 4 * ty]);
+            const float4 q0 = *reinterpret_cast<const float4 *>(&Us[jj][4 * tx]);
+            const float4 q1 = *reinterpret_cast<const float4 *>(&Us[jj][64 + 4 * tx]);
+            const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float b[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+            for (int r = 0; r < 8; ++r)
+#pragma unroll
+                for (int c = 0; c < 8; ++c) acc[r][c] = __fmaf_rn(a[r], b[c], acc[r][c]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        const int64_t n = n0 + (r < 4 ? 4 * ty + r : 64 + 4 * ty + (r - 4));
+        if (n >= N) continue;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float4 *dst = reinterpret_cast<float4 *>(Wf + n * K + k0 + 64 * h + 4 * tx);
+            float4 v = *dst;
+            v.x = __fsub_rn(v.x, acc[r][4 * h + 0]);
+            v.y = __fsub_rn(v.y, acc[r][4 * h + 1]);
+            v.z = __fsub_rn(v.z, acc[r][4 * h + 2]);
+            v.w = __fsub_rn(v.w, acc[r][4 * h + 3]);
+            *dst = v;
+        }
+    }
+}
+
+// H[j][j] += percdamp * mean(diag H); one CTA of 1024 threads, fixed-order sum.
+__global__ void __launch_bounds__(1024) gptq_damp(float *__restrict__ H, int64_t K, float percdamp) {
+    __shared__ double red[32];
+    double v = 0.0;
+    for (int64_t j = threadIdx.x; j < K; j += 1024) v += static_cast<double>(H[j * K + j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    __shared__ float lam;
+    if (threadIdx.x == 0) {
+        double s = 0.0;
+        for (int q = 0; q < 32; ++q) s += red[q];
+        lam = __fmul_rn(percdamp, __double2float_rn(s / static_cast<double>(K)));
+    }
+    __syncthreads();
+    for (int64_t j = threadIdx.x; j < K; j += 1024) H[j * K + j] = __fadd_rn(H[j * K + j], lam);
+}
+
+size_t up256(size_t v) { return (v + 255) & ~size_t(255); }
+
+struct LoopLayout {
+    size_t wf, err, total;
+};
+
+LoopLayout loop_layout(int64_t K, int64_t N, size_t at) {
+    LoopLayout L;
+    L.wf = at;
+    L.err = up256(L.wf + sizeof(float) * size_t(N) * size_t(K));
+    L.total = up256(L.err + sizeof(float) * size_t(N) * kBlock);
+    return L;
+}
+
+int column_loop(const void *W, int wt, int64_t K, int64_t N, int sym, const float *U,
+                uint8_t *packed, float *scales, float *zeros, unsigned char *ws,
+                const LoopLayout &L, cudaStream_t stream) {
+    DeviceInfo di;
+    int st = device_info(&di);
+    if (st != W4_OK) return st;
+    float *Wf = reinterpret_cast<float *>(ws + L.wf);
+    float *Err = reinterpret_cast<float *>(ws + L.err);
+    const int64_t n8 = N * K / 8;
+    const int64_t want = (n8 + 255) / 256, cap = int64_t(8) * di.sm_count;
+    gptq_widen<<<static_cast<unsigned>(want < cap ? want : cap), 256, 0, stream>>>(
+        static_cast<const uint16_t *>(W), wt, n8, Wf);
+    const unsigned row_ctas = static_cast<unsigned>((N + 7) / 8);
+    const unsigned tile_rows = static_cast<unsigned>((N + kLT - 1) / kLT);
+    for (int64_t b0 = 0; b0 < K; b0 += kBlock) {
+        if (sym)
+            gptq_block<1><<<row_ctas, 256, 0, stream>>>(Wf, U, N, K, b0, packed, scales, zeros, Err);
+        else
+            gptq_block<0><<<row_ctas, 256, 0, stream>>>(Wf, U, N, K, b0, packed, scales, zeros, Err);
+        const int64_t rest = K - b0 - kBlock;
+        if (rest > 0)
+            gptq_lazy<<<dim3(static_cast<unsigned>(rest / kLT), tile_rows), 256, 0, stream>>>(
+                Wf, Err, U, N, K, b0);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail("GPTQ column loop launch", e);
+    }
+    return W4_OK;
+}
+
+const char *shape_problem(int64_t K, int64_t N, int group) {
+    if (K <= 0 || N <= 0) return "need K, N >= 1";
+    if (group != kBlock) return "group must be 128";
+    if (K % kBlock != 0) return "K must be a multiple of 128";
+    if (K > 65536) return "K must be at most 65536";
+    if (N >= (int64_t(1) << 31) || N > (int64_t(1) << 40) / K) return "N * K too large";
+    return nullptr;
+}
+
+struct FullLayout {
+    size_t h, work, info, loop_at, total;
+    LoopLayout loop;
+};
+
+FullLayout full_layout(int64_t K, int64_t N) {
+    FullLayout F;
+    F.h = 0;
+    F.work = up256(sizeof(float) * size_t(K) * size_t(K));
+    F.info = up256(F.work + solver_work_bytes(K));
+    F.loop_at = up256(F.info + 256);
+    F.loop = loop_layout(K, N, F.loop_at);
+    F.total = F.loop.total;
+    return F;
+}
+
+}  // namespace
+}  // namespace w4
+
+using w4::set_error;
+
+extern "C" size_t w4_gptq_quantize_workspace_bytes(int64_t K, int64_t N, int group) {
+    if (w4::shape_problem(K, N, group)) return 0;
+    return w4::loop_layout(K, N, 0).total;
+}
+
+extern "C" int w4_gptq_quantize(const void *W, int wt, int64_t K, int64_t N, int group, int sym,
+                                const float *U, uint8_t *packed, float *scales, float *zeros,
+                                void *workspace, size_t workspace_bytes, void *stream) {
+    const char *fn = "w4_gptq_quantize";
+    if (wt != W4_F16 && wt != W4_BF16) return set_error(W4_ERR_INVALID_ARG, fn, "bad dtype");
+    if (const char *why = w4::shape_problem(K, N, group))
+        return set_error(group != 128 && group > 0 ? W4_ERR_UNSUPPORTED : W4_ERR_INVALID_ARG, fn, why);
+    if (!W || !U || !packed || !scales || !zeros || !workspace)
+        return set_error(W4_ERR_INVALID_ARG, fn, "null pointer");
+    const w4::LoopLayout L = w4::loop_layout(K, N, 0);
+    if (workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return set_error(W4_ERR_INVALID_ARG, fn,
+                         "workspace not 256-byte aligned or smaller than "
+                         "w4_gptq_quantize_workspace_bytes");
+    if (!w4::aligned16(W) || !w4::aligned16(U) || !w4::aligned16(packed) ||
+        !w4::aligned16(scales) || !w4::aligned16(zeros))
+        return set_error(W4_ERR_UNSUPPORTED, fn, "pointers must be 16-byte aligned");
+    return w4::column_loop(W, wt, K, N, sym, U, packed, scales, zeros,
+                           static_cast<unsigned char *>(workspace), L,
+                           static_cast<cudaStream_t>(stream));
+}
+
+extern "C" size_t w4_gptq_workspace_bytes(int64_t Mc, int64_t K, int64_t N, int group) {
+    if (Mc <= 0 || Mc >= (int64_t(1) << 31) || w4::shape_problem(K, N, group)) return 0;
+    return w4::full_layout(K, N).total;
+}
+
+extern "C" int w4_gptq(const void *W, const void *X, int xt, int64_t Mc, int64_t K, int64_t N,
+                       int group, int sym, float percdamp, uint8_t *packed, float *scales,
+                       float *zeros, float *U_out, void *workspace, size_t workspace_bytes,
+                       void *stream) {
+    const char *fn = "w4_gptq";
+    if (xt != W4_F16 && xt != W4_BF16) return set_error(W4_ERR_INVALID_ARG, fn, "bad dtype");
+    if (const char *why = w4::shape_problem(K, N, group))
+        return set_error(group != 128 && group > 0 ? W4_ERR_UNSUPPORTED : W4_ERR_INVALID_ARG, fn, why);
+    if (Mc <= 0 || Mc >= (int64_t(1) << 31)) return set_error(W4_ERR_INVALID_ARG, fn, "need 1 <= Mc < 2^31");
+    if (!(percdamp >= 0.0f && percdamp <= 1.0f))
+        return set_error(W4_ERR_INVALID_ARG, fn, "percdamp must lie in [0, 1]");
+    if (!W || !X || !packed || !scales || !zeros || !workspace)
+        return set_error(W4_ERR_INVALID_ARG, fn, "null pointer");
+    const w4::FullLayout F = w4::full_layout(K, N);
+    if (workspace_bytes < F.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return set_error(W4_ERR_INVALID_ARG, fn,
+                         "workspace not 256-byte aligned or smaller than w4_gptq_workspace_bytes");
+    if (!w4::aligned16(W) || !w4::aligned16(X) || !w4::aligned16(packed) ||
+        !w4::aligned16(scales) || !w4::aligned16(zeros) || (U_out && !w4::aligned16(U_out)))
+        return set_error(W4_ERR_UNSUPPORTED, fn, "pointers must be 16-byte aligned");
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float *H = reinterpret_cast<float *>(ws + F.h);
+    // 1. H = 2 X^T X: column-major, the K x Mc matrix X (ld K) times its transpose
+    int st = w4::blas_gemm_f32("w4_gptq (Hessian)", false, true, static_cast<int>(K),
+                               static_cast<int>(K), static_cast<int>(Mc), 2.0f, X, xt,
+                               static_cast<int>(K), X, xt, static_cast<int>(K), 0.0f, H,
+                               static_cast<int>(K), s);
+    if (st != W4_OK) return st;
+    // 2. damping
+    w4::gptq_damp<<<1, 1024, 0, s>>>(H, K, percdamp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return w4::cuda_fail("gptq_damp launch", e);
+    // 3. U, the upper Cholesky factor of H^-1 (in place)
+    st = w4::solver_inverse_factor(fn, H, static_cast<int>(K), ws + F.work, w4::solver_work_bytes(K),
+                                   reinterpret_cast<int *>(ws + F.info), s);
+    if (st != W4_OK) return st;
+    if (U_out) {
+        e = cudaMemcpyAsync(U_out, H, sizeof(float) * size_t(K) * size_t(K), cudaMemcpyDeviceToDevice, s);
+        if (e != cudaSuccess) return w4::cuda_fail("copy of U", e);
+    }
+    // 4. the column loop
+    return w4::column_loop(W, xt, K, N, sym, H, packed, scales, zeros, ws, F.loop, s);
+}

@@ -59,4 +59,19 @@ int launch_decode(const void *X, int xt, int64_t M, const uint8_t *packed, const
 int launch_prefill(const void *X, int xt, int64_t M, const uint8_t *packed, const float *scales,
                    const float *zeros, int64_t K, int64_t N, void *Y, cudaStream_t stream);
 
+// ---- NVIDIA libraries for plain dense linear algebra (w4_libs.cu) ----
+// C [m x n] fp32 (column-major, ldc) = alpha * op(A) op(B) + beta * C with
+// 16-bit A and B (types W4_F16 / W4_BF16), fp32 accumulation (cuBLAS GemmEx).
+int blas_gemm_f32(const char *fn, bool trans_a, bool trans_b, int m, int n, int k, float alpha,
+                  const void *A, int at, int lda, const void *B, int bt, int ldb, float beta,
+                  float *C, int ldc, cudaStream_t stream);
+// Work bytes reserved for solver_inverse_factor on an n x n matrix.
+size_t solver_work_bytes(int64_t n);
+// In place: H (n x n fp32, symmetric) -> the upper Cholesky factor U of H^-1
+// in row-major order (only k >= j valid).  Synchronizes `stream` once to read
+// the three factorization statuses (info_dev: 3 ints of device memory);
+// W4_ERR_INVALID_ARG if H is not positive definite.
+int solver_inverse_factor(const char *fn, float *H, int n, void *work, size_t work_bytes,
+                          int *info_dev, cudaStream_t stream);
+
 }  // namespace w4
