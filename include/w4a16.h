@@ -214,7 +214,7 @@ int w4_awq_search(const void *W, const void *X, int xt, int64_t Mc, int64_t K, i
 /*
  * w4_gptq_workspace_bytes / w4_gptq_quantize_workspace_bytes -- device
  * scratch bytes of w4_gptq and w4_gptq_quantize (0 for a shape they reject):
- * about 4 K^2 + 4 N K + 512 N bytes (w4_gptq) and 4 N K + 512 N (the loop).
+ * about 8 K^2 + 4 N K + 512 N bytes (w4_gptq) and 4 N K + 512 N (the loop).
  */
 size_t w4_gptq_workspace_bytes(int64_t Mc, int64_t K, int64_t N, int group);
 size_t w4_gptq_quantize_workspace_bytes(int64_t K, int64_t N, int group);
@@ -232,10 +232,11 @@ size_t w4_gptq_quantize_workspace_bytes(int64_t K, int64_t N, int group);
  *              (the usual 0.01; the pages give none).
  *   Outputs: packed / scales / zeros in the w4_quantize layout (w4a16_gemm
  *   consumes them unchanged); U_out nullable [K][K] fp32: the factor used
- *   (row-major, upper triangle; the strictly lower part is unspecified).
+ *   (row-major, upper triangular, zeros below the diagonal).
  *   Steps: H in fp32 (cuBLAS GEMM, fp32 accumulation); U = the upper
- *   Cholesky factor of H^-1 (cuSOLVER potrf, potri, potrf in fp32); then the
- *   column loop of w4_gptq_quantize.  The call synchronizes `stream` once,
+ *   Cholesky factor of H^-1 in fp32 (cuSOLVER: the Cholesky factor Lr of
+ *   the index-reversed H, then U = reversed(Lr^-1)); then the column loop of
+ *   w4_gptq_quantize.  The call synchronizes `stream` once,
  *   after the factorization, to read its status: W4_ERR_INVALID_ARG if the
  *   damped Hessian is not positive definite (e.g. X all zero with damping).
  *   The first call on a device opens libcublas.so.12 and libcusolver.so.11

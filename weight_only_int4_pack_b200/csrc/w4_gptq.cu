@@ -13,8 +13,9 @@
 // One call of w4_gptq, on the caller's stream:
 //   1. H = 2 X^T X in fp32 (cuBLAS GEMM, fp32 accumulation);
 //   2. damping: H_jj += percdamp * mean(diag H) (one CTA, fixed-order sum);
-//   3. U = upper Cholesky factor of H^-1 (cuSOLVER potrf, potri, potrf);
-//      the stream is synchronized once here to read the factorization status;
+//   3. U = upper Cholesky factor of H^-1 (cuSOLVER: Cholesky of the
+//      index-reversed H and a triangular inverse, see w4_libs.cu); the stream
+//      is synchronized once here to read the factorization status;
 //   4. the column loop (also alone as w4_gptq_quantize, given U):
 //      gptq_widen: Wf = fp32 copy of W;
 //      per 128-column block b (block = group):
@@ -28,7 +29,8 @@
 //          element as one fp32 fma chain over the block's 128 columns in
 //          order followed by one subtraction (a SIMT tile GEMM whose
 //          per-element order is fixed, so the result is reproducible bit for
-//          bit; 128 x 128 output tiles, 8 x 8 per thread).
+//          bit; 128 x 128 output tiles, 8 x 8 per thread, operand chunks
+//          double-buffered in shared memory).
 // Rows are independent given U: every decision of row n depends only on W[n]
 // and U, so the parallelism is over rows (block step) and over rows x later
 // columns (lazy update).  Outputs use the w4_quantize layout, so w4a16_gemm
@@ -163,46 +165,58 @@ __global__ void __launch_bounds__(256) gptq_block(float *__restrict__ Wf, const 
 // element acc = fma(Err[n][j], U[b0+j][k], acc) for j = 0, 1, ..., 127 from
 // acc = 0, then Wf = Wf - acc.  Tile 128 rows x 128 columns, 256 threads,
 // thread (ty, tx) owns rows {4ty..4ty+3, 64+4ty..64+4ty+3} and the same
-// pattern of columns.
+// pattern of columns.  The block's 128 columns go through shared memory in
+// chunks of kLJ, double-buffered: the next chunk is loaded into registers
+// while the current one is multiplied.
 __global__ void __launch_bounds__(256) gptq_lazy(float *__restrict__ Wf, const float *__restrict__ Err,
                                                  const float *__restrict__ U, int64_t N, int64_t K,
                                                  int64_t b0) {
-    __shared__ __align__(16) float Es[kLJ][kLT];
-    __shared__ __align__(16) float Us[kLJ][kLT];
+    __shared__ __align__(16) float Es[2][kLJ][kLT];
+    __shared__ __align__(16) float Us[2][kLJ][kLT];
     const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
     const int64_t n0 = static_cast<int64_t>(blockIdx.y) * kLT;
     const int64_t k0 = b0 + kBlock + static_cast<int64_t>(blockIdx.x) * kLT;
+    // this thread's share of a chunk: Err row er, columns eh..eh+7; U row uj, columns uc..uc+7
+    const int er = t >> 1, eh = (t & 1) * 8, uj = t >> 4, uc = (t & 15) * 8;
+    const bool erow_ok = n0 + er < N;
+    const float4 *esrc = reinterpret_cast<const float4 *>(Err + (n0 + er) * kBlock + eh);
+    const float4 *usrc = reinterpret_cast<const float4 *>(U + (b0 + uj) * K + k0 + uc);
+    float4 e0, e1, u0, u1;
+    auto fetch = [&](int j0) {
+        const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+        e0 = erow_ok ? esrc[j0 / 4] : zero;
+        e1 = erow_ok ? esrc[j0 / 4 + 1] : zero;
+        const float4 *u = usrc + static_cast<int64_t>(j0) * (K / 4);
+        u0 = u[0];
+        u1 = u[1];
+    };
+    auto stash = [&](int buf) {
+        Es[buf][eh + 0][er] = e0.x; Es[buf][eh + 1][er] = e0.y;
+        Es[buf][eh + 2][er] = e0.z; Es[buf][eh + 3][er] = e0.w;
+        Es[buf][eh + 4][er] = e1.x; Es[buf][eh + 5][er] = e1.y;
+        Es[buf][eh + 6][er] = e1.z; Es[buf][eh + 7][er] = e1.w;
+        *reinterpret_cast<float4 *>(&Us[buf][uj][uc]) = u0;
+        *reinterpret_cast<float4 *>(&Us[buf][uj][uc + 4]) = u1;
+    };
     float acc[8][8];
 #pragma unroll
     for (int r = 0; r < 8; ++r)
 #pragma unroll
         for (int c = 0; c < 8; ++c) acc[r][c] = 0.0f;
 
-    for (int j0 = 0; j0 < kBlock; j0 += kLJ) {
-        {   // Es[jj][r] = Err[n0 + r][j0 + jj]: thread t loads row t / 2, 8 columns
-            const int r = t >> 1, h = (t & 1) * 8;
-            float4 e0 = make_float4(0.f, 0.f, 0.f, 0.f), e1 = e0;
-            if (n0 + r < N) {
-                const float4 *src = reinterpret_cast<const float4 *>(Err + (n0 + r) * kBlock + j0 + h);
-                e0 = src[0];
-                e1 = src[1];
-            }
-            Es[h + 0][r] = e0.x; Es[h + 1][r] = e0.y; Es[h + 2][r] = e0.z; Es[h + 3][r] = e0.w;
-            Es[h + 4][r] = e1.x; Es[h + 5][r] = e1.y; Es[h + 6][r] = e1.z; Es[h + 7][r] = e1.w;
-        }
-        {   // Us[jj][c] = U[b0 + j0 + jj][k0 + c]: thread t loads row t / 16, 8 columns
-            const int jj = t >> 4, c = (t & 15) * 8;
-            const float4 *src = reinterpret_cast<const float4 *>(U + (b0 + j0 + jj) * K + k0 + c);
-            *reinterpret_cast<float4 *>(&Us[jj][c]) = src[0];
-            *reinterpret_cast<float4 *>(&Us[jj][c + 4]) = src[1];
-        }
-        __syncthreads();
+    fetch(0);
+    stash(0);
+    __syncthreads();
+#pragma unroll 1
+    for (int ch = 0; ch < kBlock / kLJ; ++ch) {
+        const int buf = ch & 1;
+        if (ch + 1 < kBlock / kLJ) fetch((ch + 1) * kLJ);
 #pragma unroll
         for (int jj = 0; jj < kLJ; ++jj) {
-            const float4 a0 = *reinterpret_cast<const float4 *>(&Es[jj][4 * ty]);
-            const float4 a1 = *reinterpret_cast<const float4 *>(&Es[jj][64 + 4 * ty]);
-            const float4 q0 = *reinterpret_cast<const float4 *>(&Us[jj][4 * tx]);
-            const float4 q1 = *reinterpret_cast<const float4 *>(&Us[jj][64 + 4 * tx]);
+            const float4 a0 = *reinterpret_cast<const float4 *>(&Es[buf][jj][4 * ty]);
+            const float4 a1 = *reinterpret_cast<const float4 *>(&Es[buf][jj][64 + 4 * ty]);
+            const float4 q0 = *reinterpret_cast<const float4 *>(&Us[buf][jj][4 * tx]);
+            const float4 q1 = *reinterpret_cast<const float4 *>(&Us[buf][jj][64 + 4 * tx]);
             const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
             const float b[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
@@ -210,6 +224,7 @@ __global__ void __launch_bounds__(256) gptq_lazy(float *__restrict__ Wf, const f
 #pragma unroll
                 for (int c = 0; c < 8; ++c) acc[r][c] = __fmaf_rn(a[r], b[c], acc[r][c]);
         }
+        if (ch + 1 < kBlock / kLJ) stash(buf ^ 1);
         __syncthreads();
     }
 #pragma unroll
@@ -301,14 +316,15 @@ const char *shape_problem(int64_t K, int64_t N, int group) {
 }
 
 struct FullLayout {
-    size_t h, work, info, loop_at, total;
+    size_t h, scratch, work, info, loop_at, total;
     LoopLayout loop;
 };
 
 FullLayout full_layout(int64_t K, int64_t N) {
     FullLayout F;
     F.h = 0;
-    F.work = up256(sizeof(float) * size_t(K) * size_t(K));
+    F.scratch = up256(sizeof(float) * size_t(K) * size_t(K));
+    F.work = up256(F.scratch + sizeof(float) * size_t(K) * size_t(K));
     F.info = up256(F.work + solver_work_bytes(K));
     F.loop_at = up256(F.info + 256);
     F.loop = loop_layout(K, N, F.loop_at);
@@ -387,7 +403,8 @@ extern "C" int w4_gptq(const void *W, const void *X, int xt, int64_t Mc, int64_t
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return w4::cuda_fail("gptq_damp launch", e);
     // 3. U, the upper Cholesky factor of H^-1 (in place)
-    st = w4::solver_inverse_factor(fn, H, static_cast<int>(K), ws + F.work, w4::solver_work_bytes(K),
+    st = w4::solver_inverse_factor(fn, H, static_cast<int>(K), reinterpret_cast<float *>(ws + F.scratch),
+                                   ws + F.work, w4::solver_work_bytes(K),
                                    reinterpret_cast<int *>(ws + F.info), s);
     if (st != W4_OK) return st;
     if (U_out) {

@@ -68,10 +68,11 @@ int blas_gemm_f32(const char *fn, bool trans_a, bool trans_b, int m, int n, int 
 // Work bytes reserved for solver_inverse_factor on an n x n matrix.
 size_t solver_work_bytes(int64_t n);
 // In place: H (n x n fp32, symmetric) -> the upper Cholesky factor U of H^-1
-// in row-major order (only k >= j valid).  Synchronizes `stream` once to read
-// the three factorization statuses (info_dev: 3 ints of device memory);
-// W4_ERR_INVALID_ARG if H is not positive definite.
-int solver_inverse_factor(const char *fn, float *H, int n, void *work, size_t work_bytes,
-                          int *info_dev, cudaStream_t stream);
+// in row-major order (zeros below the diagonal); scratch is another n x n
+// fp32 buffer.  Synchronizes `stream` once to read the factorization statuses
+// (info_dev: 2 ints of device memory); W4_ERR_INVALID_ARG if H is not
+// positive definite.
+int solver_inverse_factor(const char *fn, float *H, int n, float *scratch, void *work,
+                          size_t work_bytes, int *info_dev, cudaStream_t stream);
 
 }  // namespace w4
