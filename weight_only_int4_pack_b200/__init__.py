@@ -127,13 +127,22 @@ def _dt(t: torch.Tensor) -> int:
 
 
 def _p(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    # ctypes turns a Python int into a void* argument (None into NULL)
+    return None if t is None else t.data_ptr()
 
 
-def _stream(stream):
-    if stream is None:
-        stream = torch.cuda.current_stream()
-    return ctypes.c_void_p(stream.cuda_stream)
+try:  # the raw handle of the current stream, without building a Stream object
+    _raw_stream = torch._C._cuda_getCurrentRawStream
+except AttributeError:  # pragma: no cover
+    _raw_stream = None
+
+
+def _stream(stream, device=None):
+    if stream is not None:
+        return stream.cuda_stream
+    if _raw_stream is not None:
+        return _raw_stream(torch.cuda.current_device() if device is None else device)
+    return torch.cuda.current_stream().cuda_stream
 
 
 def _check_dev(*ts):
@@ -218,24 +227,33 @@ class Workspace:
 _default_ws = {}
 
 
+_ws_need = {}
+
+
 def w4a16_gemm_into(X, packed, scales, zeros, Y, group=128, workspace=None, stream=None):
     """Y [M][N] = X [M][K] * dequant(packed, scales, zeros)^T into caller-provided Y."""
     _check_dev(X, packed, scales, zeros, Y)
     M, K = X.shape
     N = packed.shape[0]
-    lib = load()
-    need = int(lib.w4a16_workspace_bytes(M, K, N, int(group)))
+    lib = _lib if _lib is not None else load()
+    key = (M, K, N, group)
+    need = _ws_need.get(key)
+    if need is None:
+        need = _ws_need[key] = int(lib.w4a16_workspace_bytes(M, K, N, int(group)))
+    dev = X.device
     if isinstance(workspace, Workspace) or workspace is None:
         wsobj = workspace
         if wsobj is None:
-            key = (X.device, (stream or torch.cuda.current_stream()).cuda_stream)
-            wsobj = _default_ws.setdefault(key, Workspace())
-        ws = wsobj.get(need, X.device)
+            skey = (dev, _stream(stream, dev.index))
+            wsobj = _default_ws.setdefault(skey, Workspace())
+        ws = wsobj.get(need, dev)
     else:
         ws = workspace
     wsz = 0 if ws is None else ws.numel() * ws.element_size()
-    st = lib.w4a16_gemm(_p(X), _dt(X), M, _p(packed), _p(scales), _p(zeros), K, N, int(group),
-                        _p(Y), _p(ws), wsz, _stream(stream))
+    st = lib.w4a16_gemm(X.data_ptr(), _dt(X), M, packed.data_ptr(), scales.data_ptr(),
+                        None if zeros is None else zeros.data_ptr(), K, N, group,
+                        Y.data_ptr(), None if ws is None else ws.data_ptr(), wsz,
+                        _stream(stream, dev.index))
     if st != W4_OK:
         raise W4Error("w4a16_gemm", st)
     return Y

@@ -19,9 +19,9 @@
 //   4. the column loop (also alone as w4_gptq_quantize, given U):
 //      gptq_widen: Wf = fp32 copy of W;
 //      per 128-column block b (block = group):
-//        gptq_block: one warp per weight row, lane l holding columns
-//          4l..4l+3 of the block: the group's scale / zero point from the
-//          row's current weights (the RTN quantizer's formulas), then for
+//        gptq_block: four lanes per weight row, each holding 32 of the
+//          block's columns: the group's scale / zero point from the row's
+//          current weights (the RTN quantizer's formulas), then for
 //          each column j in order: code, err_j = (w_j - (u_j - z) s) / U_jj,
 //          w_k = fma(-err_j, U_jk, w_k) for the block's k > j; writes the
 //          packed codes, scale, zero point and err[n][0..127];
@@ -85,7 +85,11 @@ __device__ __forceinline__ int code_of(float w, float s, float z) {
     return static_cast<int>(fminf(fmaxf(rintf(__fadd_rn(__fdiv_rn(w, s), z)), 0.0f), 15.0f));
 }
 
-// One warp per weight row n; block b0 .. b0 + 127 of the row.
+// Four lanes per weight row (eight rows per warp): lane quarter q of a row
+// holds the block's columns 32q .. 32q+31 in registers.  Each column step is
+// computed by the row's four lanes only (a warp advances eight rows per
+// instruction), the owner of column j broadcasts w_j within its four lanes,
+// and every lane updates its own later columns with predicated fmas.
 template <int SYM>
 __global__ void __launch_bounds__(256) gptq_block(float *__restrict__ Wf, const float *__restrict__ U,
                                                   int64_t N, int64_t K, int64_t b0,
@@ -94,68 +98,87 @@ __global__ void __launch_bounds__(256) gptq_block(float *__restrict__ Wf, const 
                                                   float *__restrict__ zeros,
                                                   float *__restrict__ Err) {
     const int lane = threadIdx.x & 31;
-    const int64_t n = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-    if (n >= N) return;  // warp-uniform
+    const int q = lane & 3;
+    const int base = lane & ~3;  // first lane of this row's four
+    const int64_t n = static_cast<int64_t>(blockIdx.x) * 64 + (threadIdx.x >> 2);
+    const bool active = n < N;  // inactive rows still take part in the shuffles
     const int64_t G = K / kBlock;
-    float *wrow = Wf + n * K + b0;
-    const float4 wv = *reinterpret_cast<const float4 *>(wrow + 4 * lane);
-    float w[4] = {wv.x, wv.y, wv.z, wv.w};
+    float w[32];
+    {
+        const float4 *src = reinterpret_cast<const float4 *>(Wf + (active ? n : 0) * K + b0 + 32 * q);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+            const float4 f = active ? src[v] : make_float4(0.f, 0.f, 0.f, 0.f);
+            w[4 * v] = f.x; w[4 * v + 1] = f.y; w[4 * v + 2] = f.z; w[4 * v + 3] = f.w;
+        }
+    }
 
-    // the group's parameters from the current weights
+    // the group's parameters from the current weights (exact min / max)
     float s, z;
     if (SYM) {
-        const float amax = warp_max(fmaxf(fmaxf(fabsf(w[0]), fabsf(w[1])), fmaxf(fabsf(w[2]), fabsf(w[3]))));
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(w[i]));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
         s = __fdiv_rn(amax, 7.0f);
         z = 8.0f;
     } else {
-        const float mn = warp_min(fminf(fminf(w[0], w[1]), fminf(w[2], w[3])));
-        const float mx = warp_max(fmaxf(fmaxf(w[0], w[1]), fmaxf(w[2], w[3])));
+        float mn = w[0], mx = w[0];
+#pragma unroll
+        for (int i = 1; i < 32; ++i) {
+            mn = fminf(mn, w[i]);
+            mx = fmaxf(mx, w[i]);
+        }
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 2));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
         s = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
         z = s == 0.0f ? 0.0f
                       : __fadd_rn(fminf(fmaxf(rintf(__fdiv_rn(-mn, s)), 0.0f), 15.0f), 0.0f);
     }
 
+    // nibble of k % 8 inside its 32-bit word: k % 8 = {0,2,4,6,1,3,5,7}[nibble]
+    constexpr int kNibble[8] = {0, 4, 1, 5, 2, 6, 3, 7};
     const float *ublk = U + b0 * K + b0;  // U[b0 + j][b0 + k] = ublk[j * K + k]
-    int my_code[4] = {0, 0, 0, 0};
-    float my_err[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    uint32_t word[4] = {0u, 0u, 0u, 0u};
+    float my_err[32];
 #pragma unroll 1
-    for (int jj = 0; jj < 32; ++jj) {
+    for (int owner = 0; owner < 4; ++owner) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int j = 4 * jj + i;
-            const float wj = __shfl_sync(0xffffffffu, w[i], jj);
+        for (int i = 0; i < 32; ++i) {
+            const int j = 32 * owner + i;
+            const float wj = __shfl_sync(0xffffffffu, w[i], base | owner);
             const int c = code_of<SYM>(wj, s, z);
             const float deq = __fmul_rn(__fsub_rn(static_cast<float>(c), z), s);
             const float e = __fdiv_rn(__fsub_rn(wj, deq), __ldg(ublk + static_cast<int64_t>(j) * K + j));
-            if (lane == jj) {
-                my_code[i] = c;
+            if (q == owner) {
+                word[i / 8] |= static_cast<uint32_t>(c) << (4 * kNibble[i % 8]);
                 my_err[i] = e;
             }
-            // columns k = 4 lane + i2 > j of the block
-            if (4 * lane + 3 > j) {
-                const float4 u4 = __ldg(reinterpret_cast<const float4 *>(ublk + static_cast<int64_t>(j) * K + 4 * lane));
-                const float uk[4] = {u4.x, u4.y, u4.z, u4.w};
+            // this lane's columns k = 32q + i2 that come after j
+            if (32 * q + 31 > j) {
+                const float4 *urow = reinterpret_cast<const float4 *>(ublk + static_cast<int64_t>(j) * K + 32 * q);
 #pragma unroll
-                for (int i2 = 0; i2 < 4; ++i2)
-                    if (4 * lane + i2 > j) w[i2] = __fmaf_rn(-e, uk[i2], w[i2]);
+                for (int v = 0; v < 8; ++v) {
+                    const float4 u4 = __ldg(urow + v);
+                    const float uk[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+                    for (int t = 0; t < 4; ++t)
+                        if (32 * q + 4 * v + t > j) w[4 * v + t] = __fmaf_rn(-e, uk[t], w[4 * v + t]);
+                }
             }
         }
     }
-
-    // codes: lanes 2m and 2m + 1 hold k = 8m..8m+3 and 8m+4..8m+7 of word m;
-    // nibble i of the word holds k = 8m + {0,2,4,6,1,3,5,7}[i]
-    const uint32_t mine = my_code[0] | (my_code[1] << 4) | (my_code[2] << 8) | (my_code[3] << 12);
-    const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
-    if ((lane & 1) == 0) {
-        const uint32_t c0 = mine & 15, c1 = (mine >> 4) & 15, c2 = (mine >> 8) & 15, c3 = (mine >> 12) & 15;
-        const uint32_t t0 = other & 15, t1 = (other >> 4) & 15, t2 = (other >> 8) & 15, t3 = (other >> 12) & 15;
-        const uint32_t word = c0 | (c2 << 4) | (t0 << 8) | (t2 << 12) | (c1 << 16) | (c3 << 20) |
-                              (t1 << 24) | (t3 << 28);
-        reinterpret_cast<uint32_t *>(packed + n * (K / 2) + b0 / 2)[lane / 2] = word;
-    }
-    reinterpret_cast<float4 *>(Err + n * kBlock)[lane] =
-        make_float4(my_err[0], my_err[1], my_err[2], my_err[3]);
-    if (lane == 0) {
+    if (!active) return;
+    reinterpret_cast<uint4 *>(packed + n * (K / 2) + b0 / 2)[q] =
+        make_uint4(word[0], word[1], word[2], word[3]);
+    float4 *edst = reinterpret_cast<float4 *>(Err + n * kBlock + 32 * q);
+#pragma unroll
+    for (int v = 0; v < 8; ++v)
+        edst[v] = make_float4(my_err[4 * v], my_err[4 * v + 1], my_err[4 * v + 2], my_err[4 * v + 3]);
+    if (q == 0) {
         scales[n * G + b0 / kBlock] = s;
         zeros[n * G + b0 / kBlock] = z;
     }
@@ -289,7 +312,7 @@ int column_loop(const void *W, int wt, int64_t K, int64_t N, int sym, const floa
     const int64_t want = (n8 + 255) / 256, cap = int64_t(8) * di.sm_count;
     gptq_widen<<<static_cast<unsigned>(want < cap ? want : cap), 256, 0, stream>>>(
         static_cast<const uint16_t *>(W), wt, n8, Wf);
-    const unsigned row_ctas = static_cast<unsigned>((N + 7) / 8);
+    const unsigned row_ctas = static_cast<unsigned>((N + 63) / 64);
     const unsigned tile_rows = static_cast<unsigned>((N + kLT - 1) / kLT);
     for (int64_t b0 = 0; b0 < K; b0 += kBlock) {
         if (sym)
