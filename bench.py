@@ -267,7 +267,11 @@ def run_ours(args, ws_, rank, local):
     copies = n_copies(sum(p.numel() + s.numel() * 8 for p, s, _ in base), l2)
     sets = [base] + [clone_set(base) for _ in range(copies - 1)]
     X = synth.activations(1, K, seed, salient_frac=c["x_salient"], dtype="f16", device=dev)
-    Ys = [torch.empty((1, N), dtype=torch.float16, device=dev) for N in Ns]
+    # the three outputs are slices of one buffer, so one copy brings a step's
+    # results to the host
+    Yall = torch.empty((1, sum(Ns)), dtype=torch.float16, device=dev)
+    offs = [sum(Ns[:i]) for i in range(len(Ns))]
+    Ys = [Yall[:, o:o + N] for o, N in zip(offs, Ns)]
     wsp = w4.Workspace()
     wsp.get(max(w4.w4a16_workspace_bytes(1, K, N) for N in Ns), dev)
 
@@ -330,14 +334,13 @@ def run_ours(args, ws_, rank, local):
 
     # e2e through the public API: pinned host X -> device, three layers, Y -> pinned host
     Xh = X.cpu().pin_memory()
-    Yh = [torch.empty((1, N), dtype=torch.float16).pin_memory() for N in Ns]
+    Yh = torch.empty((1, sum(Ns)), dtype=torch.float16).pin_memory()
     Xd = torch.empty_like(X)
 
     def step_e2e(i):
         Xd.copy_(Xh, non_blocking=True)
         step_eager(i % copies, Xd)
-        for Y, yh in zip(Ys, Yh):
-            yh.copy_(Y, non_blocking=True)
+        Yh.copy_(Yall, non_blocking=True)
 
     e2e_steps = min(args.steps, 2000)
     e2e_ms_local, _ = timed(step_e2e, e2e_steps, args.warmup)

@@ -64,18 +64,6 @@ __global__ void __launch_bounds__(256) gptq_widen(const uint16_t *__restrict__ W
     }
 }
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
-}
-
-__device__ __forceinline__ float warp_min(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
-}
-
 // Stored code of w under (s, z): sym  u = clamp(rne(w / s), -7, 7) + 8;
 // asym u = clamp(rne(fl(w / s) + z), 0, 15); a zero scale gives u = z.
 template <int SYM>
@@ -85,11 +73,19 @@ __device__ __forceinline__ int code_of(float w, float s, float z) {
     return static_cast<int>(fminf(fmaxf(rintf(__fadd_rn(__fdiv_rn(w, s), z)), 0.0f), 15.0f));
 }
 
+// Shared-memory position of U[b0 + j][b0 + c] in gptq_block: rows of kUPitch
+// floats, with 4 floats of padding after every 32 columns so that the four
+// lane quarters' 16-byte reads of one row fall in different banks.
+constexpr int kUPitch = kBlock + 16;
+constexpr int kUSmemBytes = kBlock * kUPitch * 4;  // 73728
+__device__ __forceinline__ int upos(int j, int c) { return j * kUPitch + c + 4 * (c / 32); }
+
 // Four lanes per weight row (eight rows per warp): lane quarter q of a row
 // holds the block's columns 32q .. 32q+31 in registers.  Each column step is
 // computed by the row's four lanes only (a warp advances eight rows per
 // instruction), the owner of column j broadcasts w_j within its four lanes,
-// and every lane updates its own later columns with predicated fmas.
+// and every lane updates its own later columns with predicated fmas; the U
+// values of each step come from the CTA's shared copy of the block.
 template <int SYM>
 __global__ void __launch_bounds__(256) gptq_block(float *__restrict__ Wf, const float *__restrict__ U,
                                                   int64_t N, int64_t K, int64_t b0,
@@ -97,6 +93,17 @@ __global__ void __launch_bounds__(256) gptq_block(float *__restrict__ Wf, const 
                                                   float *__restrict__ scales,
                                                   float *__restrict__ zeros,
                                                   float *__restrict__ Err) {
+    // the block's 128 x 128 part of U, staged once per CTA (padded rows, see kUPitch)
+    extern __shared__ __align__(16) float ush[];
+    {
+        const float *ublk = U + b0 * K + b0;  // U[b0 + j][b0 + k] = ublk[j * K + k]
+        for (int e = threadIdx.x; e < kBlock * kBlock / 4; e += blockDim.x) {
+            const int j = e / (kBlock / 4), c = 4 * (e % (kBlock / 4));
+            *reinterpret_cast<float4 *>(ush + upos(j, c)) =
+                __ldg(reinterpret_cast<const float4 *>(ublk + static_cast<int64_t>(j) * K + c));
+        }
+    }
+    __syncthreads();
     const int lane = threadIdx.x & 31;
     const int q = lane & 3;
     const int base = lane & ~3;  // first lane of this row's four
@@ -141,7 +148,6 @@ __global__ void __launch_bounds__(256) gptq_block(float *__restrict__ Wf, const 
 
     // nibble of k % 8 inside its 32-bit word: k % 8 = {0,2,4,6,1,3,5,7}[nibble]
     constexpr int kNibble[8] = {0, 4, 1, 5, 2, 6, 3, 7};
-    const float *ublk = U + b0 * K + b0;  // U[b0 + j][b0 + k] = ublk[j * K + k]
     uint32_t word[4] = {0u, 0u, 0u, 0u};
     float my_err[32];
 #pragma unroll 1
@@ -152,17 +158,17 @@ __global__ void __launch_bounds__(256) gptq_block(float *__restrict__ Wf, const 
             const float wj = __shfl_sync(0xffffffffu, w[i], base | owner);
             const int c = code_of<SYM>(wj, s, z);
             const float deq = __fmul_rn(__fsub_rn(static_cast<float>(c), z), s);
-            const float e = __fdiv_rn(__fsub_rn(wj, deq), __ldg(ublk + static_cast<int64_t>(j) * K + j));
+            const float e = __fdiv_rn(__fsub_rn(wj, deq), ush[upos(j, j)]);
             if (q == owner) {
                 word[i / 8] |= static_cast<uint32_t>(c) << (4 * kNibble[i % 8]);
                 my_err[i] = e;
             }
             // this lane's columns k = 32q + i2 that come after j
             if (32 * q + 31 > j) {
-                const float4 *urow = reinterpret_cast<const float4 *>(ublk + static_cast<int64_t>(j) * K + 32 * q);
+                const float4 *urow = reinterpret_cast<const float4 *>(ush + upos(j, 32 * q));
 #pragma unroll
                 for (int v = 0; v < 8; ++v) {
-                    const float4 u4 = __ldg(urow + v);
+                    const float4 u4 = urow[v];
                     const float uk[4] = {u4.x, u4.y, u4.z, u4.w};
 #pragma unroll
                     for (int t = 0; t < 4; ++t)
@@ -308,6 +314,19 @@ int column_loop(const void *W, int wt, int64_t K, int64_t N, int sym, const floa
     if (st != W4_OK) return st;
     float *Wf = reinterpret_cast<float *>(ws + L.wf);
     float *Err = reinterpret_cast<float *>(ws + L.err);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return set_error(W4_ERR_CUDA, "cudaGetDevice", nullptr);
+    static bool attr_done[64] = {};
+    if (!attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(gptq_block<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kUSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gptq_block<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kUSmemBytes);
+        if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(gptq_block smem)", e);
+        attr_done[dev] = true;
+    }
     const int64_t n8 = N * K / 8;
     const int64_t want = (n8 + 255) / 256, cap = int64_t(8) * di.sm_count;
     gptq_widen<<<static_cast<unsigned>(want < cap ? want : cap), 256, 0, stream>>>(
@@ -316,9 +335,11 @@ int column_loop(const void *W, int wt, int64_t K, int64_t N, int sym, const floa
     const unsigned tile_rows = static_cast<unsigned>((N + kLT - 1) / kLT);
     for (int64_t b0 = 0; b0 < K; b0 += kBlock) {
         if (sym)
-            gptq_block<1><<<row_ctas, 256, 0, stream>>>(Wf, U, N, K, b0, packed, scales, zeros, Err);
+            gptq_block<1><<<row_ctas, 256, kUSmemBytes, stream>>>(Wf, U, N, K, b0, packed, scales,
+                                                                 zeros, Err);
         else
-            gptq_block<0><<<row_ctas, 256, 0, stream>>>(Wf, U, N, K, b0, packed, scales, zeros, Err);
+            gptq_block<0><<<row_ctas, 256, kUSmemBytes, stream>>>(Wf, U, N, K, b0, packed, scales,
+                                                                 zeros, Err);
         const int64_t rest = K - b0 - kBlock;
         if (rest > 0)
             gptq_lazy<<<dim3(static_cast<unsigned>(rest / kLT), tile_rows), 256, 0, stream>>>(
