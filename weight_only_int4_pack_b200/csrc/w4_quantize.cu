@@ -73,6 +73,38 @@ __device__ __forceinline__ uint32_t pack8(const uint32_t b[8]) {
     return x01 | (x23 << 4) | (x45 << 8) | (x67 << 12);
 }
 
+// Packed pairs of fp32 (the f32x2 instructions of sm_100a: one instruction,
+// two independent IEEE operations rounded to nearest even, exactly as the
+// scalar forms).
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void upk2(uint64_t v, float &a, float &b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
 // Codes of eight weights with the group's s (>= FLT_MIN), r = rcp_rn(s) and
 // zero point zp (0 for symmetric, which then adds 8 through the magic).
 //
@@ -86,24 +118,31 @@ __device__ __forceinline__ uint32_t pack8(const uint32_t b[8]) {
 // range round to the clamp bound either way, so clamping y first is exact
 // (rne is monotone and 0, 15 are integers).  Symmetric groups need no clamp:
 // s >= amax/7 * (1 - 2^-24) keeps |y| < 7.5.
+// The arithmetic runs on pairs (f32x2): y, m = y + magic and d = y - (m - magic).
 template <bool SYM>
 __device__ __forceinline__ bool codes_fast(const float w[8], float r, float zp, uint32_t bits[8]) {
     bool near = false;
     const float magic = SYM ? kMagic + 8.0f : kMagic;
+    const uint64_t r2 = pk2(r, r), z2 = pk2(zp, zp), g2 = pk2(magic, magic);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        float y;
+    for (int p = 0; p < 4; ++p) {
+        const uint64_t w2 = pk2(w[2 * p], w[2 * p + 1]);
+        uint64_t y2;
         if (SYM) {
-            y = __fmul_rn(w[j], r);
+            y2 = mul2(w2, r2);
         } else {
-            y = __fmaf_rn(w[j], r, zp);
-            y = fminf(fmaxf(y, 0.0f), 15.0f);
+            float y0, y1;
+            upk2(fma2(w2, r2, z2), y0, y1);
+            y2 = pk2(fminf(fmaxf(y0, 0.0f), 15.0f), fminf(fmaxf(y1, 0.0f), 15.0f));
         }
-        const float m = __fadd_rn(y, magic);
-        const float rq = __fsub_rn(m, magic);
-        const float d = __fsub_rn(y, rq);
-        near |= fabsf(d) > 0.5f - kDelta;
-        bits[j] = __float_as_uint(m);  // 0x4B4000uu, uu = code
+        const uint64_t m2 = add2(y2, g2);
+        float d0, d1, m0, m1;
+        upk2(sub2(y2, sub2(m2, g2)), d0, d1);
+        near |= fabsf(d0) > 0.5f - kDelta;
+        near |= fabsf(d1) > 0.5f - kDelta;
+        upk2(m2, m0, m1);
+        bits[2 * p] = __float_as_uint(m0);  // 0x4B4000uu, uu = code
+        bits[2 * p + 1] = __float_as_uint(m1);
     }
     return near;
 }
@@ -171,7 +210,8 @@ quantize_kernel(const uint16_t *__restrict__ W, int64_t K, int64_t N,
                 load8<WT>(raw[i], w);
                 if (FOLD) {
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) w[j] = __fmul_rn(w[j], cs[j]);
+                    for (int j = 0; j < 8; j += 2)
+                        upk2(mul2(pk2(w[j], w[j + 1]), pk2(cs[j], cs[j + 1])), w[j], w[j + 1]);
                 }
                 float s, zp;
                 if (SYM) {
