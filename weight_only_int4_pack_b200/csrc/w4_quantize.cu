@@ -15,12 +15,14 @@
 // rounding boundary (k + 1/2).  The bound on |fast - exact| is derived in the
 // comment of `codes_fast`.
 //
-// Work layout: a CTA of 128 threads owns a strip of 1024 consecutive k and
-// walks down RT rows of it.  Thread t covers k = 8t..8t+7 of the strip: one
-// 16-byte load of eight 16-bit weights and one 32-bit packed word per row.
-// GROUP/8 adjacent lanes form one group and reduce its amax (or min/max)
-// with butterfly shuffles.  A warp writes 128 contiguous bytes of codes per
-// row; the strip's scales and zeros of a row are contiguous too.
+// Work layout: a CTA of 128 threads owns a strip of 2048 consecutive k and
+// walks down RT rows of it.  Thread t covers k = 16t..16t+15 of the strip:
+// two 16-byte loads of sixteen 16-bit weights and two 32-bit packed words per
+// row, so the per-group work (the reduction, the scale and zero point, the
+// reciprocal) is shared by sixteen weights per thread.  GROUP/16 adjacent
+// lanes form one group and reduce its amax (or min/max) with butterfly
+// shuffles.  A warp writes 256 contiguous bytes of codes per row; the strip's
+// scales and zeros of a row are contiguous too.
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -32,7 +34,8 @@ namespace w4 {
 namespace {
 
 constexpr int kThreads = 128;
-constexpr int kStripK = kThreads * 8;  // 1024 k per CTA tile
+constexpr int kPer = 16;                // consecutive k per thread
+constexpr int kStripK = kThreads * kPer;  // 2048 k per CTA tile
 constexpr int kRowsPerTile = 32;
 constexpr int kRowUnroll = 4;
 
@@ -170,7 +173,7 @@ quantize_kernel(const uint16_t *__restrict__ W, int64_t K, int64_t N,
                 const float *__restrict__ col_scale, uint32_t *__restrict__ packed,
                 float *__restrict__ scales, float *__restrict__ zeros, int64_t tiles_k,
                 int64_t tiles) {
-    constexpr int LPG = GROUP / 8;  // lanes per group (4, 8, 16 or 32)
+    constexpr int LPG = GROUP / kPer;  // lanes per group (2, 4, 8 or 16)
     const int t = threadIdx.x;
     const int lane = t & 31;
     const int64_t G = K / GROUP;
@@ -178,46 +181,51 @@ quantize_kernel(const uint16_t *__restrict__ W, int64_t K, int64_t N,
     for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
         const int64_t kb = tile % tiles_k;
         const int64_t rb = tile / tiles_k;
-        const int64_t k = kb * kStripK + 8 * t;
+        const int64_t k = kb * kStripK + kPer * t;
         const bool valid_k = k < K;  // uniform over each group since K % GROUP == 0
-        float cs[8];
+        float cs[kPer];
         if (FOLD) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) cs[j] = 1.0f;
+            for (int j = 0; j < kPer; ++j) cs[j] = 1.0f;
             if (valid_k) {
-                const float4 c0 = __ldg(reinterpret_cast<const float4 *>(col_scale + k));
-                const float4 c1 = __ldg(reinterpret_cast<const float4 *>(col_scale + k + 4));
-                cs[0] = c0.x; cs[1] = c0.y; cs[2] = c0.z; cs[3] = c0.w;
-                cs[4] = c1.x; cs[5] = c1.y; cs[6] = c1.z; cs[7] = c1.w;
+#pragma unroll
+                for (int v = 0; v < kPer / 4; ++v) {
+                    const float4 c = __ldg(reinterpret_cast<const float4 *>(col_scale + k) + v);
+                    cs[4 * v] = c.x; cs[4 * v + 1] = c.y; cs[4 * v + 2] = c.z; cs[4 * v + 3] = c.w;
+                }
             }
         }
         const int64_t row0 = rb * kRowsPerTile;
         for (int rr = 0; rr < kRowsPerTile; rr += kRowUnroll) {
             if (row0 + rr >= N) break;  // uniform over the CTA
-            uint4 raw[kRowUnroll];
+            uint4 raw[kRowUnroll][2];
 #pragma unroll
             for (int i = 0; i < kRowUnroll; ++i) {
                 const int64_t row = row0 + rr + i;
-                raw[i] = make_uint4(0, 0, 0, 0);
-                if (valid_k && row < N)
-                    raw[i] = __ldcs(reinterpret_cast<const uint4 *>(W + row * K + k));
+                raw[i][0] = raw[i][1] = make_uint4(0, 0, 0, 0);
+                if (valid_k && row < N) {
+                    const uint4 *src = reinterpret_cast<const uint4 *>(W + row * K + k);
+                    raw[i][0] = __ldcs(src);
+                    raw[i][1] = __ldcs(src + 1);
+                }
             }
 #pragma unroll
             for (int i = 0; i < kRowUnroll; ++i) {
                 const int64_t row = row0 + rr + i;
                 if (row >= N) break;  // uniform
-                float w[8];
-                load8<WT>(raw[i], w);
+                float w[kPer];
+                load8<WT>(raw[i][0], w);
+                load8<WT>(raw[i][1], w + 8);
                 if (FOLD) {
 #pragma unroll
-                    for (int j = 0; j < 8; j += 2)
+                    for (int j = 0; j < kPer; j += 2)
                         upk2(mul2(pk2(w[j], w[j + 1]), pk2(cs[j], cs[j + 1])), w[j], w[j + 1]);
                 }
                 float s, zp;
                 if (SYM) {
                     float a = fabsf(w[0]);
 #pragma unroll
-                    for (int j = 1; j < 8; ++j) a = fmaxf(a, fabsf(w[j]));
+                    for (int j = 1; j < kPer; ++j) a = fmaxf(a, fabsf(w[j]));
 #pragma unroll
                     for (int off = LPG / 2; off >= 1; off >>= 1)
                         a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
@@ -226,7 +234,7 @@ quantize_kernel(const uint16_t *__restrict__ W, int64_t K, int64_t N,
                 } else {
                     float mn = w[0], mx = w[0];
 #pragma unroll
-                    for (int j = 1; j < 8; ++j) {
+                    for (int j = 1; j < kPer; ++j) {
                         mn = fminf(mn, w[j]);
                         mx = fmaxf(mx, w[j]);
                     }
@@ -241,19 +249,22 @@ quantize_kernel(const uint16_t *__restrict__ W, int64_t K, int64_t N,
                     if (s != 0.0f)
                         zp = __fadd_rn(fminf(fmaxf(rintf(__fdiv_rn(-mn, s)), 0.0f), 15.0f), 0.0f);
                 }
-                uint32_t bits[8];
+                uint32_t bits[kPer];
                 if (s == 0.0f) {
                     const uint32_t u = 0x4B400000u | static_cast<uint32_t>(zp);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) bits[j] = u;
+                    for (int j = 0; j < kPer; ++j) bits[j] = u;
                 } else {
                     const float r = __frcp_rn(s);
                     const bool fast_ok = s >= FLT_MIN;
-                    bool near = codes_fast<SYM>(w, r, SYM ? 0.0f : zp, bits);
-                    if (near || !fast_ok) codes_exact<SYM>(w, s, zp, bits);
+                    const bool near0 = codes_fast<SYM>(w, r, SYM ? 0.0f : zp, bits);
+                    const bool near1 = codes_fast<SYM>(w + 8, r, SYM ? 0.0f : zp, bits + 8);
+                    if (near0 || !fast_ok) codes_exact<SYM>(w, s, zp, bits);
+                    if (near1 || !fast_ok) codes_exact<SYM>(w + 8, s, zp, bits + 8);
                 }
                 if (valid_k) {
-                    packed[(row * K + k) >> 3] = pack8(bits);
+                    reinterpret_cast<uint2 *>(packed)[(row * K + k) >> 4] =
+                        make_uint2(pack8(bits), pack8(bits + 8));
                     if ((lane % LPG) == 0) {
                         const int64_t gi = row * G + k / GROUP;
                         scales[gi] = s;
