@@ -10,7 +10,8 @@
 // and §4.6 FP8 (scale = max|x| / 448, cast to E4M3).
 //
 // Per-tensor quantization is two passes over the tensor: amax_kernel (a
-// max-reduction of |v|, one atomicMax on the float's bits per CTA -- the
+// max-reduction of |v| -- per-column maxima of |a|, the column op applied once
+// per column -- with one atomicMax on the float's bits per CTA -- the
 // bits of non-negative floats order like the values, and max does not depend
 // on the order, so the result is exact and deterministic), then quant8_kernel
 // (every thread derives the scale from amax; CTA 0 publishes it).  Column
@@ -65,20 +66,39 @@ __device__ __forceinline__ unsigned block_max_bits(unsigned b, unsigned *red) {
 }
 
 // *amax_bits = max(*amax_bits, bits of max |v|) over the tensor (zeroed before).
+// Thread (x, y) owns the 8-column word x of the rows y, y + gridDim.y, ... and
+// keeps the largest |a| of each of its columns; the column op is applied once
+// per column at the end.  That is exact: the correctly rounded product or
+// quotient by a fixed factor is monotone in |a|, so the largest |fl(a op c)|
+// of a column is fl(max |a| op |c|).
 template <int XT, int OP>
-__global__ void __launch_bounds__(256) amax_kernel(const uint16_t *__restrict__ A, int64_t n8,
+__global__ void __launch_bounds__(256) amax_kernel(const uint16_t *__restrict__ A, int64_t rows,
                                                    int64_t K, const float *__restrict__ col,
                                                    unsigned *__restrict__ amax_bits) {
     __shared__ unsigned red[8];
-    float m = 0.0f;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
-         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        float v[8];
-        load_v8<XT, OP>(A, col, i, K, v);
+    const int64_t w = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t words = K / 8;
+    float m[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
+    for (int j = 0; j < 8; ++j) m[j] = 0.0f;
+    if (w < words) {
+        for (int64_t r = blockIdx.y; r < rows; r += gridDim.y) {
+            float f[8];
+            widen8<XT>(__ldg(reinterpret_cast<const uint4 *>(A + r * K) + w), f);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) m[j] = fmaxf(m[j], fabsf(f[j]));
+        }
     }
-    const unsigned b = block_max_bits(__float_as_uint(m), red);
+    float best = 0.0f;
+    if (w < words) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float v = m[j];
+            if (OP != W8_COL_NONE) v = fabsf(col_apply<OP>(v, fabsf(__ldg(col + 8 * w + j))));
+            best = fmaxf(best, v);
+        }
+    }
+    const unsigned b = block_max_bits(__float_as_uint(best), red);
     if (threadIdx.x == 0) atomicMax(amax_bits, b);
 }
 
@@ -183,7 +203,14 @@ int quantize_t(const uint16_t *A, int64_t rows, int64_t K, const float *col, flo
     const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
     cudaError_t e = cudaMemsetAsync(scale + 1, 0, sizeof(float), stream);
     if (e != cudaSuccess) return cuda_fail("cudaMemsetAsync(amax)", e);
-    amax_kernel<XT, OP><<<grid, 256, 0, stream>>>(A, n8, K, col, reinterpret_cast<unsigned *>(scale + 1));
+    const int64_t words = K / 8;
+    const unsigned gx = static_cast<unsigned>((words + 255) / 256);
+    int64_t gy = cap / gx;
+    if (gy < 1) gy = 1;
+    if (gy > rows) gy = rows;
+    if (gy > 65535) gy = 65535;
+    amax_kernel<XT, OP><<<dim3(gx, static_cast<unsigned>(gy)), 256, 0, stream>>>(
+        A, rows, K, col, reinterpret_cast<unsigned *>(scale + 1));
     quant8_kernel<XT, OP, FMT><<<grid, 256, 0, stream>>>(A, n8, K, col, scale, q);
     return cuda_status(cudaGetLastError());
 }
