@@ -227,7 +227,8 @@ size_t w4_gptq_quantize_workspace_bytes(int64_t K, int64_t N, int group);
  *
  *   W          [N][K] fp16 or bf16 (xt), the weight; X [Mc][K] the same dtype,
  *              the layer's calibration activations.
- *   group      must be 128 (the GPTQ block); K % 128 == 0; sym as w4_quantize.
+ *   group      must be 128 (the GPTQ block); K % 128 == 0, K <= 65536,
+ *              N <= 8388480; sym as w4_quantize.
  *   percdamp   damping in [0, 1]: H = 2 X^T X + percdamp * mean(diag) * I
  *              (the usual 0.01; the pages give none).
  *   Outputs: packed / scales / zeros in the w4_quantize layout (w4a16_gemm

@@ -239,6 +239,7 @@ def test_gptq_argument_checks(lib):
     assert call(group=64) == 2         # group must be 128
     assert call(Mc=0) == 1
     assert call(N=0) == 1
+    assert call(N=65535 * 128 + 1) == 1   # beyond the lazy update's grid
     assert call(xt=4) == 1
     assert call(pd=F(-0.5)) == 1
     assert call(W=None) == 1

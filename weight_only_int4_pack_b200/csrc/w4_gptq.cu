@@ -355,7 +355,8 @@ const char *shape_problem(int64_t K, int64_t N, int group) {
     if (group != kBlock) return "group must be 128";
     if (K % kBlock != 0) return "K must be a multiple of 128";
     if (K > 65536) return "K must be at most 65536";
-    if (N >= (int64_t(1) << 31) || N > (int64_t(1) << 40) / K) return "N * K too large";
+    if (N > int64_t(65535) * kLT) return "N must be at most 8388480";  // lazy-update grid rows
+    if (N > (int64_t(1) << 40) / K) return "N * K too large";
     return nullptr;
 }
 
