@@ -55,6 +55,11 @@ int launch_decode(const void *X, int xt, int64_t M, const uint8_t *packed, const
                   const float *zeros, int64_t K, int64_t N, void *Y, void *workspace,
                   size_t workspace_bytes, cudaStream_t stream);
 
+// decode path for M <= 8, K <= 4096 (warp-level tensor-core GEMV); needs no workspace
+bool gemv_supported(int64_t M, int64_t K);
+int launch_gemv(const void *X, int xt, int64_t M, const uint8_t *packed, const float *scales,
+                const float *zeros, int64_t K, int64_t N, void *Y, cudaStream_t stream);
+
 // prefill path, M > 32 (tcgen05)
 int launch_prefill(const void *X, int xt, int64_t M, const uint8_t *packed, const float *scales,
                    const float *zeros, int64_t K, int64_t N, void *Y, cudaStream_t stream);
