@@ -92,13 +92,16 @@ int w4_quantize(const void *W, int wt, int64_t K, int64_t N, int group, int sym,
 
 /*
  * w4a16_workspace_bytes -- scratch bytes w4a16_gemm needs for this shape
- * (0 when it needs none).  The workspace holds per-tile arrival counters
+ * (0 when it needs none: 1 <= M <= 8 with K <= 4096, and shapes whose row
+ * blocks are not split).  The workspace holds per-tile arrival counters
  * (a fixed area at its start) and split-K partial sums.  It must be
  * zero-filled once before its first use; every w4a16_gemm call leaves the
  * counter area zero again when its work completes and fully rewrites the
  * partials it reads, so one workspace serves any number of calls of any
  * shapes issued one after another on ONE stream.  Calls that may overlap on
- * the GPU (other streams) need separate workspaces.
+ * the GPU (other streams) need separate workspaces.  A call whose bounded
+ * wait ran out (w4_device_status reports W4_ERR_TIMEOUT) may stop partway and
+ * leave counters armed: zero-fill the workspace again before reusing it.
  */
 size_t w4a16_workspace_bytes(int64_t M, int64_t K, int64_t N, int group);
 
@@ -114,16 +117,19 @@ size_t w4a16_workspace_bytes(int64_t M, int64_t K, int64_t N, int group);
  *   fp32 (the integer (u - zero) is exact in the 16-bit operand type; the
  *   group scale multiplies the fp32 partial sum of its group) and rounded
  *   once to the output dtype.
- *   M <= 32 runs the decode path (persistent stream-K tensor-core GEMV);
- *   larger M runs the tcgen05 path (TMA-staged X, dequantized W tiles in
- *   shared memory, accumulators in tensor memory).
- *   The decode path is launched with programmatic dependent launch: it may
- *   start while the preceding kernel of the stream finishes, and it starts
- *   streaming `packed` before that kernel has completed (X, scales, zeros, Y
- *   and the workspace are touched only after).  So `packed` must not be
- *   written by the immediately preceding kernel if that kernel itself allows
- *   early dependent launch (the kernels of this library that write `packed`
- *   do not).
+ *   1 <= M <= 8 with K <= 4096 runs the small-M decode GEMV (one CTA per SM,
+ *   whole rows, warp-level tensor-core MMAs, no workspace); other M <= 32
+ *   run the persistent stream-K decode path on tcgen05; larger M runs the
+ *   tcgen05 prefill path (TMA-staged X, dequantized W tiles in shared
+ *   memory, accumulators in tensor memory).
+ *   The decode paths are launched with programmatic dependent launch: they
+ *   may start while the preceding kernel of the stream finishes, and they
+ *   start streaming the weights before that kernel has completed (the
+ *   tcgen05 decode path `packed` only; the small-M GEMV `packed`, `scales`
+ *   and `zeros`).  X, Y and the workspace are touched only after.  So the
+ *   weights must not be written by the immediately preceding kernel if that
+ *   kernel itself allows early dependent launch (the kernels of this library
+ *   that write them do not).
  *   workspace / workspace_bytes: at least w4a16_workspace_bytes(M, K, N, group)
  *   bytes of device memory prepared as described there (may be NULL when
  *   that size is 0); a smaller workspace returns W4_ERR_INVALID_ARG.
@@ -151,7 +157,12 @@ int w4a16_gemm(const void *X, int xt, int64_t M, const uint8_t *packed, const fl
  *   All calls on a device share the one array: calls that may overlap on the
  *   GPU (other streams, other host threads) race and give wrong results.
  *   The first call on each device looks up the array's device address with
- *   that device current; make that first call before any stream capture.
+ *   that device current, which may also load the library's device code and
+ *   the 4 MiB array onto the device (CUDA loads modules lazily) -- a step
+ *   that can allocate device memory and synchronize.  Make that first call
+ *   as a warm-up, outside any latency-critical path and before any stream
+ *   capture.  Shapes whose decode kernel uses no scratch space (see
+ *   w4a16_workspace_bytes) never touch the array.
  */
 int w4a16_gemm_noalloc(const void *X, int xt, int64_t M, const uint8_t *packed,
                        const float *scales, const float *zeros, int64_t K, int64_t N, int group,

@@ -1,9 +1,18 @@
 """The C ABI of libw4a16.so, checked without a GPU: it builds, loads, exports
 every function include/w4a16.h declares, and rejects invalid arguments with
-the documented status before anything reaches the device."""
+the documented status before anything reaches the device.
+
+The argument checks pass fake, never-dereferenced addresses.  They only ever
+run in a process that sees no GPU: where a GPU is visible, this module's tests
+are skipped in-process and re-run as a child pytest with
+CUDA_VISIBLE_DEVICES="", so that even a regression in the host-side checks
+could not launch a kernel on those addresses (the call would fail with
+W4_ERR_CUDA instead)."""
 import ctypes
 import os
 import re
+import subprocess
+import sys
 
 import pytest
 
@@ -11,6 +20,32 @@ import weight_only_int4_pack_b200 as w4
 from weight_only_int4_pack_b200 import build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _gpu_visible():
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False
+
+
+GPU_VISIBLE = _gpu_visible()
+
+
+@pytest.fixture(autouse=True)
+def _no_visible_gpu(request):
+    if GPU_VISIBLE and request.node.name != "test_module_in_a_process_without_gpu":
+        pytest.skip("fake-address checks run in a child process without a visible GPU")
+
+
+@pytest.mark.skipif(not GPU_VISIBLE, reason="runs in-process here: no GPU is visible")
+def test_module_in_a_process_without_gpu():
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-p", "no:cacheprovider",
+                        os.path.abspath(__file__)], cwd=ROOT, env=env, capture_output=True,
+                       text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
 
 
 @pytest.fixture(scope="module")

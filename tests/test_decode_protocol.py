@@ -198,3 +198,39 @@ def test_model_detects_a_deadlock():
         assert run_cta(KS, *rs[0], 3, 7) is not None
     finally:
         Bar = orig
+
+
+def counter_protocol(contrib, counters, stored, abort_after=None):
+    """The split row block hand-over of `decode_kernel`, one (row block, warp)
+    counter: each contributing CTA stores its partial, then arrives with an
+    atomic add; the arrival that reads count - 1 adds the partials (those
+    stored so far) and re-arms the counter to 0.  `abort_after` = number of
+    contributors that arrive before the rest stop (a bounded wait ran out).
+    Returns the partial sum written to Y, or None if nobody wrote it."""
+    written = None
+    c = len(contrib)
+    for i, part in enumerate(contrib):
+        if abort_after is not None and i >= abort_after:
+            break
+        stored.append(part)
+        prev = counters[0]
+        counters[0] += 1
+        if prev == c - 1:
+            written = sum(stored)
+            counters[0] = 0
+    return written
+
+
+def test_counters_after_a_timeout_need_a_cleared_workspace():
+    """A call that stops partway (a bounded wait ran out, W4_ERR_TIMEOUT)
+    leaves the counter nonzero; the next call on the same workspace then
+    writes no row or a wrong one.  Zero-filling the workspace again, as the
+    header asks after W4_ERR_TIMEOUT, restores correct results."""
+    parts = [1.0, 2.0, 4.0]
+    ws = [0]
+    assert counter_protocol(parts, ws, []) == 7.0 and ws[0] == 0  # normal calls re-arm
+    assert counter_protocol(parts, ws, [], abort_after=2) is None
+    assert ws[0] == 2  # left armed by the aborted call
+    assert counter_protocol(parts, ws, []) != 7.0  # stale counter: wrong or missing
+    ws[0] = 0  # the workspace zero-filled again
+    assert counter_protocol(parts, ws, []) == 7.0

@@ -125,3 +125,97 @@ def test_beats_rtn_on_calibration_data(sym):
     Xv, Wv = vals(X), vals(W)
     err = lambda p, s, z: np.linalg.norm((oracle.dequant(p, s, None if sym else z, K, 128) - Wv) @ Xv.T)
     assert err(p, s, z) < 0.6 * err(pr, sr, zr)
+
+
+def exact_case(N, K, sym, seed, group=128):
+    """Weights and a factor U on which every fp32 and fp64 operation of the
+    GPTQ update is exact, so the oracle's fp32 loop and the pages' fp64
+    recursion must give the same codes and scales bit for bit.
+
+    Per group: two anchor columns hold the group's extremes (-0.5 and 7/16,
+    or +-7/16 symmetric), so its scale is 1/16 and its zero point 8; every
+    other weight is a multiple of 2^-10 well inside that range.  Columns are
+    sources (their errors are pushed onward) or sinks (they receive errors and
+    push none): U is upper triangular with diagonal 1/2, 1 or 2 and a few
+    off-diagonal entries +-1/8, +-1/16 from sources to later sinks, in the
+    same and in later 128-column blocks.  Errors are then multiples of 2^-11,
+    updates of 2^-15, and no sink leaves the anchors' range."""
+    rng = np.random.default_rng(seed)
+    W = np.round(rng.uniform(-0.35, 0.3, (N, K)) * 1024) / 1024
+    role = rng.integers(0, 2, K)  # 1 = source
+    for g in range(K // group):
+        a = g * group + rng.choice(group, 2, replace=False)
+        W[:, a[0]] = -7 / 16 if sym else -0.5
+        W[:, a[1]] = 7 / 16
+        role[a] = 2  # anchors: neither updated nor pushing (their error is 0 anyway)
+    U = np.diag(rng.choice([0.5, 1.0, 2.0], K))
+    for k in range(K):
+        if role[k] != 0:
+            continue
+        srcs = [j for j in range(k) if role[j] == 1]
+        for j in rng.choice(srcs, min(3, len(srcs)), replace=False) if srcs else []:
+            U[j, k] = rng.choice([0.125, -0.125, 0.0625, -0.0625])
+    return W, U
+
+
+@pytest.mark.parametrize("sym", [True, False])
+@pytest.mark.parametrize("N,K,seed", [(6, 256, 1), (10, 384, 2), (4, 512, 3), (16, 256, 4)])
+def test_exact_against_the_pages_update(N, K, seed, sym):
+    Wv, U = exact_case(N, K, sym, seed)
+    W16 = torch.from_numpy(Wv).to(torch.float16)
+    assert np.array_equal(vals(W16), Wv)  # the weights are exact in fp16
+    p, s, z = oracle.gptq_quantize(bits(W16), oracle.F16, U.astype(np.float32), 128, sym)
+    # the pages' recursion with H^-1 = U^T U given directly (no damping)
+    codes_ref, scales_ref = pages_update(Wv, U.T @ U, 128, sym)
+    np.testing.assert_array_equal(unpack(p, K), codes_ref)
+    np.testing.assert_array_equal(s.astype(np.float64), scales_ref)
+    assert np.all(s == np.float32(1 / 16))
+    # some errors really crossed columns and blocks (the case is not trivial)
+    pr, sr, zr = oracle.quantize(bits(W16), oracle.F16, 128, sym)
+    assert not np.array_equal(p, pr)
+
+
+def pages_update(Wv, Hinv, group, sym, mistake=None):
+    """The pages' recursion (as obs_reference) with H^-1 given directly, fp64.
+    `mistake` plants one error for the sensitivity check: "sign" (errors
+    added instead of subtracted), "nodiv" (no division by [H_F^-1]_jj),
+    "stale" (column j never removed from H_F^-1)."""
+    N, K = Wv.shape
+    Hinv = Hinv.copy()
+    W = Wv.copy()
+    codes = np.zeros((N, K), np.int64)
+    scales = np.zeros((N, K // group))
+    for j in range(K):
+        if j % group == 0:
+            blk = W[:, j:j + group].astype(np.float32)
+            if sym:
+                s = np.abs(blk).max(1) / np.float32(7)
+                z = np.full(N, 8.0, np.float32)
+            else:
+                mn, mx = blk.min(1), blk.max(1)
+                s = (mx - mn) / np.float32(15)
+                z = np.clip(np.round(-mn / s), 0, 15).astype(np.float32)
+            scales[:, j // group] = s
+        wj = W[:, j].astype(np.float32)
+        u = np.clip(np.round(wj / s), -7, 7) + 8 if sym else np.clip(np.round(wj / s + z), 0, 15)
+        codes[:, j] = u
+        q = (u - z.astype(np.float64)) * s.astype(np.float64)
+        delta = (W[:, j] - q) / (1.0 if mistake == "nodiv" else Hinv[j, j])
+        upd = np.outer(delta, Hinv[j, j + 1:])
+        W[:, j + 1:] += upd if mistake == "sign" else -upd
+        if mistake != "stale":
+            Hinv = Hinv - np.outer(Hinv[:, j], Hinv[j, :]) / Hinv[j, j]
+    return codes, scales
+
+
+@pytest.mark.parametrize("mistake", ["sign", "nodiv", "stale"])
+def test_exact_case_catches_planted_mistakes(mistake):
+    """The exact construction is sensitive to the update it checks: each
+    planted mistake in the pages' recursion changes the codes."""
+    Wv, U = exact_case(8, 256, False, 5)
+    W16 = torch.from_numpy(Wv).to(torch.float16)
+    p, s, z = oracle.gptq_quantize(bits(W16), oracle.F16, U.astype(np.float32), 128, False)
+    good, _ = pages_update(Wv, U.T @ U, 128, False)
+    bad, _ = pages_update(Wv, U.T @ U, 128, False, mistake)
+    np.testing.assert_array_equal(unpack(p, 256), good)
+    assert not np.array_equal(good, bad)

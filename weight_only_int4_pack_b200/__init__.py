@@ -170,9 +170,20 @@ def w4_abi_version() -> int:
     return int(load().w4_abi_version())
 
 
+# Bumped when a bounded wait is seen to have run out: a kernel that stopped
+# partway may have left the arrival counters of a decode workspace armed, so
+# every Workspace zero-fills itself again before its next use.
+_ws_epoch = [0]
+
+
 def w4_device_status(reset: bool = True) -> int:
-    """Status word set by kernels whose bounded waits ran out (synchronizes)."""
-    return int(load().w4_device_status(int(bool(reset))))
+    """Status word set by kernels whose bounded waits ran out (synchronizes).
+    On W4_ERR_TIMEOUT every Workspace of this module is zero-filled again
+    before its next use, as include/w4a16.h asks."""
+    st = int(load().w4_device_status(int(bool(reset))))
+    if st == W4_ERR_TIMEOUT:
+        _ws_epoch[0] += 1
+    return st
 
 
 def w4_selftest_wait_timeout(timeout_us: int = 1000, stream=None) -> None:
@@ -210,17 +221,23 @@ def w4a16_workspace_bytes(M: int, K: int, N: int, group: int = 128) -> int:
 
 
 class Workspace:
-    """A zero-filled device workspace that grows on demand (one per stream)."""
+    """A zero-filled device workspace that grows on demand (one per stream).
+    Zero-filled again after a bounded wait ran out (see w4_device_status)."""
 
     def __init__(self, device=None):
         self.buf = None
         self.device = device
+        self.epoch = _ws_epoch[0]
 
     def get(self, nbytes: int, device):
         if nbytes == 0:
             return None
         if self.buf is None or self.buf.numel() < nbytes or self.buf.device != device:
             self.buf = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
+            self.epoch = _ws_epoch[0]
+        elif self.epoch != _ws_epoch[0]:
+            self.buf.zero_()
+            self.epoch = _ws_epoch[0]
         return self.buf
 
 
