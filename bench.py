@@ -48,11 +48,12 @@ METRIC = "W4A16 g128 dequant-GEMM TB/s (decode) & TFLOPS (prefill) vs B200 roofl
 GROUP = 128
 
 # DRAM traffic of one decode launch (M=1, K=4096, N=12288: the dominant
-# kernel of the step) from one ncu capture (dram__bytes_read.sum +
-# dram__bytes_write.sum; profiles/decode_kernel_m1_k4096_n12288.md), valid
-# only for the kernel source it was taken on: reported as null once that
-# source has changed.
-DECODE_TRAFFIC = {"bytes": 28391168, "source_sha256_16": "79c24eff2796b109"}
+# kernel of the step, gemv_kernel of csrc/w4_gemv.cu) from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum; profiles/gemv_kernel_m1_k4096_n12288.md),
+# valid only for the kernel source it was taken on: reported as null once
+# that source has changed.
+DECODE_SRC = "w4_gemv.cu"
+DECODE_TRAFFIC = {"bytes": None, "source_sha256_16": ""}
 
 
 # ---------------------------------------------------------------------------- helpers
@@ -322,11 +323,11 @@ def run_ours(args, ws_, rank, local):
         b = decode_bytes(1, K, N, c["sym"])
         per_layer.append({"N": N, "us": kms * 1e3, "bytes": b, "gbs": b / (kms * 1e-3) / 1e9})
     dom = max(per_layer, key=lambda d: d["us"])
-    src = os.path.join(ROOT, "weight_only_int4_pack_b200", "csrc", "w4_decode.cu")
+    src = os.path.join(ROOT, "weight_only_int4_pack_b200", "csrc", DECODE_SRC)
     cur = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] if os.path.exists(src) else ""
     traffic = DECODE_TRAFFIC["bytes"] if (cur == DECODE_TRAFFIC["source_sha256_16"]
                                           and dom["N"] == 12288) else None
-    roof = {"bound": "hbm", "kernel": "decode_kernel (w4a16_gemm, M=1)",
+    roof = {"bound": "hbm", "kernel": "gemv_kernel (w4a16_gemm, M=1)",
             "achieved": round(dom["gbs"], 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": round(dom["gbs"] / pk["hbm_gbs"], 4), "traffic": traffic,
             "peak_source": pk["source"], "bytes_per_launch": dom["bytes"],
@@ -358,12 +359,13 @@ def run_ours(args, ws_, rank, local):
             if args.sections == "all"
             else set())
         del graphs, layer_graphs, gblock
+        cpu_ok = args.n_gpus == 1 and not args.no_cpu
         if "decode_small_m" in want:
-            sections["decode_small_m"] = section_small_m(w4, dev, l2, pk)
+            sections["decode_small_m"] = section_small_m(w4, dev, l2, pk, cpu_ok)
         if "prefill" in want:
-            sections["prefill"] = section_prefill(w4, dev, pk)
+            sections["prefill"] = section_prefill(w4, dev, pk, cpu_ok)
         if "quantize" in want:
-            sections["quantize_7b_stack"] = section_quantize(w4, dev, pk)
+            sections["quantize_7b_stack"] = section_quantize(w4, dev, pk, cpu_ok)
         if "awq" in want:
             sections["awq_search"] = section_awq(w4, dev, pk)
         if "w8a8" in want:
@@ -380,7 +382,7 @@ def run_ours(args, ws_, rank, local):
                 gpu_launches=launches_per_step * args.steps)
 
 
-def section_small_m(w4, dev, l2, pk):
+def section_small_m(w4, dev, l2, pk, cpu=False):
     c = synth.DECODE_SMALLM
     K, N = c["K"], c["N"]
     base = [make_layer(w4, N, K, c["sym"], c["seed"], 4, std=c["std"])]
@@ -405,11 +407,15 @@ def section_small_m(w4, dev, l2, pk):
                     "tflops": round(2 * M * N * K / (kms * 1e-3) / 1e12, 2),
                     "frac_hbm": round(gbs / pk["hbm_gbs"], 4)})
         del g, ws
-    return {"workload": f"decode M in {list(c['Ms'])}, K={K}, N={N}, symmetric g128 fp16",
-            "bound": "hbm", "peak_gbs": pk["hbm_gbs"], "copies": copies, "per_m": out}
+    res = {"workload": f"decode M in {list(c['Ms'])}, K={K}, N={N}, symmetric g128 fp16",
+           "bound": "hbm", "peak_gbs": pk["hbm_gbs"], "copies": copies, "per_m": out}
+    if cpu:
+        p, sc, _ = host_layers([sets[0][0]])[0]
+        res["cpu_baseline"] = cpu_small_m(p, sc, K, N, c)
+    return res
 
 
-def section_prefill(w4, dev, pk):
+def section_prefill(w4, dev, pk, cpu=False):
     c = synth.PREFILL
     M, K, N = c["M"], c["K"], c["N"]
     p, s, z = make_layer(w4, N, K, c["sym"], c["seed"], 4, dtype="bf16", std=c["std"])
@@ -437,12 +443,16 @@ def section_prefill(w4, dev, pk):
             times.append(e0.elapsed_time(e1))
     kms = statistics.median(times)
     tf = 2 * M * N * K / (kms * 1e-3) / 1e12
-    return {"workload": f"prefill M={M} K={K} N={N} asymmetric g128 bf16", "bound": "tensor",
-            "us": round(kms * 1e3, 1), "tflops": round(tf, 1), "peak_tflops": pk["bf16_tflops"],
-            "frac": round(tf / pk["bf16_tflops"], 4), "l2": "flushed between launches"}
+    res = {"workload": f"prefill M={M} K={K} N={N} asymmetric g128 bf16", "bound": "tensor",
+           "us": round(kms * 1e3, 1), "tflops": round(tf, 1), "peak_tflops": pk["bf16_tflops"],
+           "frac": round(tf / pk["bf16_tflops"], 4), "l2": "flushed between launches"}
+    if cpu:
+        hp, hs, hz = host_layers([(p, s, z)])[0]
+        res["cpu_baseline"] = cpu_prefill(X.cpu(), hp, hs, hz, M, K, N)
+    return res
 
 
-def section_quantize(w4, dev, pk):
+def section_quantize(w4, dev, pk, cpu=False):
     c = synth.STACK_7B
     Xcal = synth.activations(c["calib_M"], 4096, c["seed"], salient_frac=c["x_salient"],
                              tensor_id=2, device=dev)
@@ -485,11 +495,16 @@ def section_quantize(w4, dev, pk):
     nw = sum(w.numel() for lw in Ws for w in lw)
     b = nw * (2 + 0.5 + 8 / GROUP)
     gbs = b / (kms * 1e-3) / 1e9
-    return {"workload": "quantize 32 x {qkv 12288x4096, o 4096x4096, gate_up 22016x4096, "
-                        "down 4096x11008}, AWQ factor folded (in=4096), asymmetric g128",
-            "bound": "hbm", "weights": nw, "ms": round(kms, 3), "gbs": round(gbs, 1),
-            "frac": round(gbs / pk["hbm_gbs"], 4), "launches": len(Ws) * 4,
-            "bytes_per_weight": 2 + 0.5 + 8 / GROUP}
+    res = {"workload": "quantize 32 x {qkv 12288x4096, o 4096x4096, gate_up 22016x4096, "
+                       "down 4096x11008}, AWQ factor folded (in=4096), asymmetric g128",
+           "bound": "hbm", "weights": nw, "ms": round(kms, 3), "gbs": round(gbs, 1),
+           "frac": round(gbs / pk["hbm_gbs"], 4), "launches": len(Ws) * 4,
+           "bytes_per_weight": 2 + 0.5 + 8 / GROUP}
+    if cpu:
+        host = [w.cpu() for w in layer]
+        del Ws, outs
+        res["cpu_baseline"] = cpu_quantize(host, cs.cpu(), c["layers"])
+    return res
 
 
 def awq_inputs(dev):
@@ -673,6 +688,123 @@ def oracle_step(layer_sets_host, Xbits, dtype):
 def host_layers(layers):
     return [(p.cpu().numpy(), s.cpu().numpy(), None if z is None else z.cpu().numpy())
             for p, s, z in layers]
+
+
+def _cpu_info():
+    import oracle
+    model = ""
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return {"cores": oracle.threads(), "nproc": os.cpu_count(), "cpu_model": model}
+
+
+def _one_core(fn):
+    """Runs fn() with the oracle on one thread; returns its result."""
+    import oracle
+    n = oracle.threads()
+    oracle.set_threads(1)
+    try:
+        return fn()
+    finally:
+        oracle.set_threads(n)
+
+
+def cpu_small_m(packed, scales, K, N, c):
+    """The oracle on the small-M decode layers (K = 8192, N = 28672,
+    symmetric): fp64 dequantization + naive fp64 product, every M in full on
+    all cores; on one core the M = 4 layer on its first 1024 weight rows,
+    scaled to the full N (labelled)."""
+    import oracle
+    info = _cpu_info()
+    out = []
+    for M in c["Ms"]:
+        X = synth.activations(M, K, c["seed"], salient_frac=c["x_salient"])
+        xb = X.contiguous().view(torch.int16).numpy().view(np.uint16)
+        t0 = time.perf_counter()
+        W2 = oracle.dequant(packed, scales, None, K, GROUP)
+        oracle.linear(xb, oracle.F16, W2)
+        el = time.perf_counter() - t0
+        b = decode_bytes(M, K, N, True)
+        out.append({"M": M, "s": round(el, 3), "gbs": round(b / el / 1e9, 3)})
+        del W2
+    X = synth.activations(4, K, c["seed"], salient_frac=c["x_salient"])
+    xb = X.contiguous().view(torch.int16).numpy().view(np.uint16)
+    rows = 1024
+
+    def one():
+        t0 = time.perf_counter()
+        Wr = oracle.dequant(packed[:rows], scales[:rows], None, K, GROUP)
+        oracle.linear(xb, oracle.F16, Wr)
+        return time.perf_counter() - t0
+    el1 = _one_core(one) * N / rows
+    return dict(info, kind="oracle", unit="GB/s", value=out[0]["gbs"], per_m=out,
+                sample="every M of the layer in full (all cores)",
+                one_core={"M": 4, "s_extrapolated": round(el1, 2),
+                          "gbs": round(decode_bytes(4, K, N, True) / el1 / 1e9, 4),
+                          "sample": f"first {rows} of {N} rows, time scaled by {N}/{rows}"})
+
+
+def cpu_prefill(X, packed, scales, zeros, M, K, N):
+    """The oracle on the prefill layer (M = 2048, K = 4096, N = 11008): fp64
+    dequantization and the naive fp64 product on a seeded sample of 256 rows of
+    X (all N), all cores; 32 of those rows on one core.  The full-size time is
+    the sample's scaled by the rows (labelled as an extrapolation)."""
+    import oracle
+    info = _cpu_info()
+    xb = X.contiguous().view(torch.int16).numpy().view(np.uint16)
+    rows = np.sort(np.random.default_rng(4).choice(M, 256, replace=False))
+    t0 = time.perf_counter()
+    What = oracle.dequant(packed, scales, zeros, K, GROUP)
+    oracle.linear(xb, oracle.BF16, What, rows=rows)
+    el = time.perf_counter() - t0
+    full = el * M / len(rows)
+    tf = 2 * M * N * K / full / 1e12
+
+    def one():
+        t0 = time.perf_counter()
+        oracle.linear(xb, oracle.BF16, What, rows=rows[:32])
+        return time.perf_counter() - t0
+    el1 = _one_core(one) * M / 32
+    return dict(info, kind="oracle", unit="TFLOP/s", value=round(tf, 6),
+                sample=f"256 of {M} rows of X, all N; full-size time extrapolated "
+                       f"({full:.1f} s) from the sample's {el:.2f} s",
+                one_core={"tflops": round(2 * M * N * K / el1 / 1e12, 7),
+                          "s_extrapolated": round(el1, 1),
+                          "sample": f"32 of {M} rows, scaled by {M}/32"})
+
+
+def cpu_quantize(layer, cs, nlayers):
+    """The oracle quantizer on the 7B stack: the seeded layer (4 projections,
+    AWQ factor folded where in = 4096, asymmetric) quantized 32 times -- the
+    same work as the GPU section's 32 layers -- on all cores; one projection
+    (o, 4096 x 4096) on one core, scaled to the stack (labelled)."""
+    import oracle
+    info = _cpu_info()
+    hb = [w.contiguous().view(torch.int16).numpy().view(np.uint16) for w in layer]
+    csn = cs.numpy().astype(np.float32)
+    nw = sum(w.size for w in hb) * nlayers
+    t0 = time.perf_counter()
+    for _ in range(nlayers):
+        for w in hb:
+            oracle.quantize(w, oracle.F16, GROUP, False, csn if w.shape[1] == 4096 else None)
+    el = time.perf_counter() - t0
+    b = nw * (2 + 0.5 + 8 / GROUP)
+    o = hb[1]
+
+    def one():
+        t0 = time.perf_counter()
+        oracle.quantize(o, oracle.F16, GROUP, False, csn)
+        return time.perf_counter() - t0
+    el1 = _one_core(one) * nw / o.size
+    return dict(info, kind="oracle", unit="GB/s", value=round(b / el / 1e9, 3), s=round(el, 2),
+                sample=f"the whole stack ({nlayers} x the seeded layer, {nw} weights)",
+                one_core={"gbs": round(b / el1 / 1e9, 4), "s_extrapolated": round(el1, 1),
+                          "sample": "the o projection (4096 x 4096), scaled to the stack"})
 
 
 def cpu_baseline(layers, X, step_bytes):

@@ -148,27 +148,48 @@ def test_values_next_to_rounding_boundaries(sym):
     assert_same(gpu_quantize(W, 128, sym, col), oracle_quantize(W, 128, sym, col), "near-boundary")
 
 
+def _fp16_magnitudes():
+    """All positive finite fp16 values, ascending (31743 of them)."""
+    allv = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16).view(np.float16)
+    allv = allv[np.isfinite(allv)]
+    return np.unique(np.abs(allv[allv != 0]))
+
+
+def _sweep_chunk(P, i0, i1):
+    """Groups [amax, x_1 .. x_127] for amax = P[i], i0 <= i < i1, whose x run
+    over every fp16 value with |x| <= amax: 0, +-P[0..i]; padded with zeros."""
+    blocks = []
+    for i in range(i0, i1):
+        xs = np.concatenate([[np.float16(0)], P[:i + 1], -P[:i + 1]])
+        ng = (xs.size + 126) // 127
+        xs = np.concatenate([xs, np.zeros(ng * 127 - xs.size, np.float16)]).reshape(ng, 127)
+        blocks.append(np.concatenate([np.full((ng, 1), P[i], np.float16), xs], axis=1))
+    W = np.concatenate(blocks)
+    pad = (-W.shape[0]) % 8  # 8 groups per row
+    W = np.concatenate([W, np.zeros((pad, 128), np.float16)]).reshape(-1, 1024)
+    return torch.from_numpy(W)
+
+
 def test_symmetric_code_map_over_all_fp16_values():
-    """Every finite fp16 x against a spread of fp16 amax values: each group is
-    [amax, x_1..x_127] with |x_i| <= amax, so the code of every x is decided
-    by the scale amax/7 alone."""
-    allv = torch.arange(0, 1 << 16, dtype=torch.int32).to(torch.int16).view(torch.float16).float()
-    allv = allv[torch.isfinite(allv)]
-    pos = torch.unique(allv.abs())
-    pos = pos[pos > 0]
-    amaxes = pos[torch.linspace(0, pos.numel() - 1, 1024).long()]
-    groups = []
-    for a in amaxes.tolist():
-        xs = allv[allv.abs() <= a]
-        nfull = (xs.numel() + 126) // 127
-        xs = torch.cat([xs, torch.zeros(nfull * 127 - xs.numel())])
-        blk = torch.cat([torch.full((nfull, 1), a), xs.view(nfull, 127)], dim=1)
-        groups.append(blk)
-    W = torch.cat(groups).to(torch.float16)
-    # 8 groups per row keeps rows long enough for the CTA strip
-    pad = (-W.shape[0]) % 8
-    W = torch.cat([W, torch.zeros(pad, 128, dtype=torch.float16)]).view(-1, 1024)
-    assert_same(gpu_quantize(W, 128, True), oracle_quantize(W, 128, True), "fp16 sweep")
+    """The symmetric scale -> code map exhaustively: every finite fp16 x
+    against every positive finite fp16 amax (about 10^9 pairs, in chunks).
+    Each group is [amax, x_1..x_127] with |x_i| <= amax, so the code of every
+    x is decided by the scale fl(amax / 7) alone; codes, packed bytes and the
+    scales are compared bit for bit with the oracle."""
+    P = _fp16_magnitudes()
+    assert P.size == 31743
+    # chunk boundaries holding about 2^26 weights each (the work of amax i
+    # grows like i)
+    cum = np.cumsum(2 * np.arange(P.size) + 3)
+    bounds = [0] + list(np.searchsorted(cum, np.arange(1, 64) * (cum[-1] / 64))) + [P.size]
+    bounds = sorted(set(int(x) for x in bounds))
+    pairs = 0
+    for i0, i1 in zip(bounds[:-1], bounds[1:]):
+        W = _sweep_chunk(P, i0, i1)
+        pairs += int(cum[i1 - 1] - (cum[i0 - 1] if i0 else 0))
+        assert_same(gpu_quantize(W, 128, True), oracle_quantize(W, 128, True),
+                    f"fp16 sweep amax {P[i0]}..{P[i1 - 1]}")
+    assert pairs > 10 ** 9
 
 
 def test_7b_layer_full_size_sampled_rows():
