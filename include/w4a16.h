@@ -24,8 +24,8 @@
  * Conventions shared by every entry point:
  *   - All array arguments are DEVICE pointers of the current CUDA device,
  *     allocated and owned by the caller; the library allocates no memory
- *     (exceptions: the first w4_awq_search or w4_gptq on a device creates
- *     cuBLAS / cuSOLVER handles there, which allocate their own workspace).
+ *     (exception: the first w4_awq_search on a device creates a cuBLAS
+ *     handle there, which allocates its own workspace).
  *     Base pointers must be 16-byte aligned (else W4_ERR_UNSUPPORTED).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *     Every call only enqueues work and returns: results are ready once the
@@ -117,16 +117,18 @@ size_t w4a16_workspace_bytes(int64_t M, int64_t K, int64_t N, int group);
  *   fp32 (the integer (u - zero) is exact in the 16-bit operand type; the
  *   group scale multiplies the fp32 partial sum of its group) and rounded
  *   once to the output dtype.
- *   1 <= M <= 8 with K <= 4096 runs the small-M decode GEMV (one CTA per SM,
- *   whole rows, warp-level tensor-core MMAs, no workspace); other M <= 32
- *   run the persistent stream-K decode path on tcgen05; larger M runs the
+ *   M = 1 with K % 512 == 0 and K <= 4096 runs the CUDA-core GEMV (one CTA
+ *   per SM, whole rows streamed per warp, no workspace); other 1 <= M <= 8
+ *   with K <= 4096 the small-M GEMV on warp-level tensor-core MMAs (whole
+ *   rows, no workspace); other M <= 32 the persistent stream-K decode path
+ *   on tcgen05; larger M runs the
  *   tcgen05 prefill path (TMA-staged X, dequantized W tiles in shared
  *   memory, accumulators in tensor memory).
  *   The decode paths are launched with programmatic dependent launch: they
  *   may start while the preceding kernel of the stream finishes, and they
  *   start streaming the weights before that kernel has completed (the
- *   tcgen05 decode path `packed` only; the small-M GEMV `packed`, `scales`
- *   and `zeros`).  X, Y and the workspace are touched only after.  So the
+ *   tcgen05 decode path `packed` only; the GEMVs `packed`, `scales` and
+ *   `zeros`).  X, Y and the workspace are touched only after.  So the
  *   weights must not be written by the immediately preceding kernel if that
  *   kernel itself allows early dependent launch (the kernels of this library
  *   that write them do not).
@@ -245,15 +247,14 @@ size_t w4_gptq_quantize_workspace_bytes(int64_t K, int64_t N, int group);
  *   Outputs: packed / scales / zeros in the w4_quantize layout (w4a16_gemm
  *   consumes them unchanged); U_out nullable [K][K] fp32: the factor used
  *   (row-major, upper triangular, zeros below the diagonal).
- *   Steps: H in fp32 (cuBLAS GEMM, fp32 accumulation); U = the upper
- *   Cholesky factor of H^-1 in fp32 (cuSOLVER: the Cholesky factor Lr of
- *   the index-reversed H, then U = reversed(Lr^-1)); then the column loop of
- *   w4_gptq_quantize.  The call synchronizes `stream` once,
- *   after the factorization, to read its status: W4_ERR_INVALID_ARG if the
- *   damped Hessian is not positive definite (e.g. X all zero with damping).
- *   The first call on a device opens libcublas.so.12 and libcusolver.so.11
- *   and creates their handles (kept until exit); a missing library returns
- *   W4_ERR_UNSUPPORTED.
+ *   Steps, all this library's kernels in fp32 with IEEE division and square
+ *   root: H = 2 X^T X (tiled GEMM, fp32 accumulation); U = the upper
+ *   Cholesky factor of H^-1 without forming H^-1 (the blocked Cholesky
+ *   factor Lr of the index-reversed H, a blocked triangular inverse, then
+ *   U = reversed(Lr^-1)); then the column loop of w4_gptq_quantize.  The call
+ *   synchronizes `stream` once, after the factorization, to read its status:
+ *   W4_ERR_INVALID_ARG if the damped Hessian is not positive definite (e.g. X
+ *   all zero with damping).  No library is called.
  *   workspace: w4_gptq_workspace_bytes bytes, 256-byte aligned, clobbered.
  */
 int w4_gptq(const void *W, const void *X, int xt, int64_t Mc, int64_t K, int64_t N, int group,

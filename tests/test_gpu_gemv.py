@@ -1,6 +1,7 @@
-"""Parity of the small-M decode path (1 <= M <= 8, K <= 4096: the
-warp-level tensor-core GEMV, no workspace) with the oracle's fp64 product,
-through the C ABI.
+"""Parity of the small-M decode paths with the oracle's fp64 product, through
+the C ABI: M = 1 with K % 512 == 0 (the CUDA-core GEMV) and every other
+1 <= M <= 8 with K <= 4096 (the warp-level tensor-core GEMV); neither takes a
+workspace.
 
 The packed weights are the oracle's own quantization of seeded weights; the
 tolerance is the W4A16 one of tests/helpers.py."""
@@ -52,10 +53,12 @@ def test_every_m(M, dtype):
     run(M, 1000, 4096, M % 2 == 0, dtype, 40 + M)
 
 
+@pytest.mark.parametrize("M", [1, 2])
 @pytest.mark.parametrize("N", [1, 2, 7, 15, 16, 17, 147, 148, 149, 296, 2371, 4101])
-def test_row_counts(N):
-    """Rows per CTA from 0 to many, partial tiles of 16 rows."""
-    run(1, N, 4096, False, "f16", N)
+def test_row_counts(N, M):
+    """Rows per CTA from 0 to many, partial batches of 4 rows (M = 1) and
+    partial tiles of 16 rows (M = 2)."""
+    run(M, N, 4096, False, "f16", N + M)
 
 
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])

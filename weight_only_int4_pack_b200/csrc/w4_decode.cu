@@ -921,7 +921,7 @@ size_t decode_counter_bytes() { return kCounterBytes; }
 
 size_t decode_workspace_bytes(int64_t M, int64_t K, int64_t N, int group) {
     (void)group;
-    if (gemv_supported(M, K)) return 0;
+    if (gemv1_supported(M, K) || gemv_supported(M, K)) return 0;
     Work w;
     size_t b = 0;
     if (make_work(M, K, N, &w, &b) != W4_OK) return 0;
@@ -931,6 +931,7 @@ size_t decode_workspace_bytes(int64_t M, int64_t K, int64_t N, int group) {
 int launch_decode(const void *X, int xt, int64_t M, const uint8_t *packed, const float *scales,
                   const float *zeros, int64_t K, int64_t N, void *Y, void *workspace,
                   size_t workspace_bytes, cudaStream_t stream) {
+    if (gemv1_supported(M, K)) return launch_gemv1(X, xt, packed, scales, zeros, K, N, Y, stream);
     if (gemv_supported(M, K))
         return launch_gemv(X, xt, M, packed, scales, zeros, K, N, Y, stream);
     Work w;

@@ -11,11 +11,11 @@
 // rows of X [Mc][K], so H = 2 X^T X is [K][K].
 //
 // One call of w4_gptq, on the caller's stream:
-//   1. H = 2 X^T X in fp32 (cuBLAS GEMM, fp32 accumulation);
+//   1. H = 2 X^T X in fp32 (this library's tiled GEMM, w4_linalg.cu);
 //   2. damping: H_jj += percdamp * mean(diag H) (one CTA, fixed-order sum);
-//   3. U = upper Cholesky factor of H^-1 (cuSOLVER: Cholesky of the
-//      index-reversed H and a triangular inverse, see w4_libs.cu); the stream
-//      is synchronized once here to read the factorization status;
+//   3. U = upper Cholesky factor of H^-1 (w4_linalg.cu: blocked Cholesky of
+//      the index-reversed H and a blocked triangular inverse); the stream is
+//      synchronized once here to read the factorization status;
 //   4. the column loop (also alone as w4_gptq_quantize, given U):
 //      gptq_widen: Wf = fp32 copy of W;
 //      per 128-column block b (block = group):
@@ -47,7 +47,7 @@ namespace {
 
 constexpr int kBlock = 128;  // GPTQ block = quantization group
 constexpr int kLT = 128;     // lazy update: output tile rows and columns
-constexpr int kLJ = 16;      // lazy update: block columns per shared-memory stage
+constexpr int kLJ = 8;       // lazy update: block columns per shared-memory stage
 
 __global__ void __launch_bounds__(256) gptq_widen(const uint16_t *__restrict__ W, int wt,
                                                   int64_t n8, float *__restrict__ Wf) {
@@ -84,30 +84,36 @@ __device__ __forceinline__ int upos(int j, int c) { return j * kUPitch + c + 4 *
 // holds the block's columns 32q .. 32q+31 in registers.  Each column step is
 // computed by the row's four lanes only (a warp advances eight rows per
 // instruction), the owner of column j broadcasts w_j within its four lanes,
-// and every lane updates its own later columns with predicated fmas; the U
-// values of each step come from the CTA's shared copy of the block.
+// and the lanes whose quarter reaches column j update all of it; the U values
+// of each step come from the CTA's shared copy of the block.  128 threads (32
+// rows) per CTA, so that the CTAs spread evenly over the SMs.
 template <int SYM>
-__global__ void __launch_bounds__(256) gptq_block(float *__restrict__ Wf, const float *__restrict__ U,
+__global__ void __launch_bounds__(128) gptq_block(float *__restrict__ Wf, const float *__restrict__ U,
                                                   int64_t N, int64_t K, int64_t b0,
                                                   uint8_t *__restrict__ packed,
                                                   float *__restrict__ scales,
                                                   float *__restrict__ zeros,
                                                   float *__restrict__ Err) {
-    // the block's 128 x 128 part of U, staged once per CTA (padded rows, see kUPitch)
+    // the block's 128 x 128 part of U, staged once per CTA (padded rows, see
+    // kUPitch), its strict lower triangle as zeros
     extern __shared__ __align__(16) float ush[];
     {
         const float *ublk = U + b0 * K + b0;  // U[b0 + j][b0 + k] = ublk[j * K + k]
         for (int e = threadIdx.x; e < kBlock * kBlock / 4; e += blockDim.x) {
             const int j = e / (kBlock / 4), c = 4 * (e % (kBlock / 4));
-            *reinterpret_cast<float4 *>(ush + upos(j, c)) =
-                __ldg(reinterpret_cast<const float4 *>(ublk + static_cast<int64_t>(j) * K + c));
+            float4 u = __ldg(reinterpret_cast<const float4 *>(ublk + static_cast<int64_t>(j) * K + c));
+            if (c < j) u.x = 0.0f;
+            if (c + 1 < j) u.y = 0.0f;
+            if (c + 2 < j) u.z = 0.0f;
+            if (c + 3 < j) u.w = 0.0f;
+            *reinterpret_cast<float4 *>(ush + upos(j, c)) = u;
         }
     }
     __syncthreads();
     const int lane = threadIdx.x & 31;
     const int q = lane & 3;
     const int base = lane & ~3;  // first lane of this row's four
-    const int64_t n = static_cast<int64_t>(blockIdx.x) * 64 + (threadIdx.x >> 2);
+    const int64_t n = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 4) + (threadIdx.x >> 2);
     const bool active = n < N;  // inactive rows still take part in the shuffles
     const int64_t G = K / kBlock;
     float w[32];
@@ -163,16 +169,19 @@ __global__ void __launch_bounds__(256) gptq_block(float *__restrict__ Wf, const 
                 word[i / 8] |= static_cast<uint32_t>(c) << (4 * kNibble[i % 8]);
                 my_err[i] = e;
             }
-            // this lane's columns k = 32q + i2 that come after j
-            if (32 * q + 31 > j) {
+            // this lane's columns k = 32q + i2 >= j (q >= owner), all of them:
+            // the staged U[j][k] is 0 for k < j, and w[j] itself is no
+            // longer read, so the columns after j get exactly their update
+            // and no predicate is needed
+            if (q >= owner) {
                 const float4 *urow = reinterpret_cast<const float4 *>(ush + upos(j, 32 * q));
 #pragma unroll
                 for (int v = 0; v < 8; ++v) {
                     const float4 u4 = urow[v];
-                    const float uk[4] = {u4.x, u4.y, u4.z, u4.w};
-#pragma unroll
-                    for (int t = 0; t < 4; ++t)
-                        if (32 * q + 4 * v + t > j) w[4 * v + t] = __fmaf_rn(-e, uk[t], w[4 * v + t]);
+                    w[4 * v] = __fmaf_rn(-e, u4.x, w[4 * v]);
+                    w[4 * v + 1] = __fmaf_rn(-e, u4.y, w[4 * v + 1]);
+                    w[4 * v + 2] = __fmaf_rn(-e, u4.z, w[4 * v + 2]);
+                    w[4 * v + 3] = __fmaf_rn(-e, u4.w, w[4 * v + 3]);
                 }
             }
         }
@@ -197,35 +206,32 @@ __global__ void __launch_bounds__(256) gptq_block(float *__restrict__ Wf, const 
 // pattern of columns.  The block's 128 columns go through shared memory in
 // chunks of kLJ, double-buffered: the next chunk is loaded into registers
 // while the current one is multiplied.
-__global__ void __launch_bounds__(256) gptq_lazy(float *__restrict__ Wf, const float *__restrict__ Err,
-                                                 const float *__restrict__ U, int64_t N, int64_t K,
-                                                 int64_t b0) {
+__global__ void __launch_bounds__(256, 2) gptq_lazy(float *__restrict__ Wf, const float *__restrict__ Err,
+                                                    const float *__restrict__ U, int64_t N, int64_t K,
+                                                    int64_t b0) {
     __shared__ __align__(16) float Es[2][kLJ][kLT];
     __shared__ __align__(16) float Us[2][kLJ][kLT];
     const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
     const int64_t n0 = static_cast<int64_t>(blockIdx.y) * kLT;
     const int64_t k0 = b0 + kBlock + static_cast<int64_t>(blockIdx.x) * kLT;
-    // this thread's share of a chunk: Err row er, columns eh..eh+7; U row uj, columns uc..uc+7
-    const int er = t >> 1, eh = (t & 1) * 8, uj = t >> 4, uc = (t & 15) * 8;
+    // this thread's share of a chunk: Err row er, block columns eh..eh+3 (a
+    // warp stores 32 consecutive rows: no bank conflicts); U row uj, columns
+    // uc..uc+3
+    const int er = t & (kLT - 1), eh = (t >> 7) * 4, uj = t >> 5, uc = (t & 31) * 4;
     const bool erow_ok = n0 + er < N;
     const float4 *esrc = reinterpret_cast<const float4 *>(Err + (n0 + er) * kBlock + eh);
     const float4 *usrc = reinterpret_cast<const float4 *>(U + (b0 + uj) * K + k0 + uc);
-    float4 e0, e1, u0, u1;
+    float4 e0, u0;
     auto fetch = [&](int j0) {
-        const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
-        e0 = erow_ok ? esrc[j0 / 4] : zero;
-        e1 = erow_ok ? esrc[j0 / 4 + 1] : zero;
-        const float4 *u = usrc + static_cast<int64_t>(j0) * (K / 4);
-        u0 = u[0];
-        u1 = u[1];
+        e0 = erow_ok ? esrc[j0 / 4] : make_float4(0.f, 0.f, 0.f, 0.f);
+        u0 = usrc[static_cast<int64_t>(j0) * (K / 4)];
     };
     auto stash = [&](int buf) {
-        Es[buf][eh + 0][er] = e0.x; Es[buf][eh + 1][er] = e0.y;
-        Es[buf][eh + 2][er] = e0.z; Es[buf][eh + 3][er] = e0.w;
-        Es[buf][eh + 4][er] = e1.x; Es[buf][eh + 5][er] = e1.y;
-        Es[buf][eh + 6][er] = e1.z; Es[buf][eh + 7][er] = e1.w;
+        Es[buf][eh + 0][er] = e0.x;
+        Es[buf][eh + 1][er] = e0.y;
+        Es[buf][eh + 2][er] = e0.z;
+        Es[buf][eh + 3][er] = e0.w;
         *reinterpret_cast<float4 *>(&Us[buf][uj][uc]) = u0;
-        *reinterpret_cast<float4 *>(&Us[buf][uj][uc + 4]) = u1;
     };
     float acc[8][8];
 #pragma unroll
@@ -256,19 +262,34 @@ __global__ void __launch_bounds__(256) gptq_lazy(float *__restrict__ Wf, const f
         if (ch + 1 < kBlock / kLJ) stash(buf ^ 1);
         __syncthreads();
     }
+    // Wf -= acc, two rows at a time: their four reads are issued before the
+    // stores (a store to Wf could alias a later read)
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        const int64_t n = n0 + (r < 4 ? 4 * ty + r : 64 + 4 * ty + (r - 4));
-        if (n >= N) continue;
+    for (int rr = 0; rr < 8; rr += 2) {
+        float4 v[2][2];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            float4 *dst = reinterpret_cast<float4 *>(Wf + n * K + k0 + 64 * h + 4 * tx);
-            float4 v = *dst;
-            v.x = __fsub_rn(v.x, acc[r][4 * h + 0]);
-            v.y = __fsub_rn(v.y, acc[r][4 * h + 1]);
-            v.z = __fsub_rn(v.z, acc[r][4 * h + 2]);
-            v.w = __fsub_rn(v.w, acc[r][4 * h + 3]);
-            *dst = v;
+        for (int u = 0; u < 2; ++u) {
+            const int r = rr + u;
+            const int64_t n = n0 + (r < 4 ? 4 * ty + r : 64 + 4 * ty + (r - 4));
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+                v[u][h] = n < N ? *reinterpret_cast<const float4 *>(Wf + n * K + k0 + 64 * h + 4 * tx)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int r = rr + u;
+            const int64_t n = n0 + (r < 4 ? 4 * ty + r : 64 + 4 * ty + (r - 4));
+            if (n >= N) continue;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float4 w = v[u][h];
+                w.x = __fsub_rn(w.x, acc[r][4 * h + 0]);
+                w.y = __fsub_rn(w.y, acc[r][4 * h + 1]);
+                w.z = __fsub_rn(w.z, acc[r][4 * h + 2]);
+                w.w = __fsub_rn(w.w, acc[r][4 * h + 3]);
+                *reinterpret_cast<float4 *>(Wf + n * K + k0 + 64 * h + 4 * tx) = w;
+            }
         }
     }
 }
@@ -331,14 +352,14 @@ int column_loop(const void *W, int wt, int64_t K, int64_t N, int sym, const floa
     const int64_t want = (n8 + 255) / 256, cap = int64_t(8) * di.sm_count;
     gptq_widen<<<static_cast<unsigned>(want < cap ? want : cap), 256, 0, stream>>>(
         static_cast<const uint16_t *>(W), wt, n8, Wf);
-    const unsigned row_ctas = static_cast<unsigned>((N + 63) / 64);
+    const unsigned row_ctas = static_cast<unsigned>((N + 31) / 32);  // 32 rows per CTA
     const unsigned tile_rows = static_cast<unsigned>((N + kLT - 1) / kLT);
     for (int64_t b0 = 0; b0 < K; b0 += kBlock) {
         if (sym)
-            gptq_block<1><<<row_ctas, 256, kUSmemBytes, stream>>>(Wf, U, N, K, b0, packed, scales,
+            gptq_block<1><<<row_ctas, 128, kUSmemBytes, stream>>>(Wf, U, N, K, b0, packed, scales,
                                                                  zeros, Err);
         else
-            gptq_block<0><<<row_ctas, 256, kUSmemBytes, stream>>>(Wf, U, N, K, b0, packed, scales,
+            gptq_block<0><<<row_ctas, 128, kUSmemBytes, stream>>>(Wf, U, N, K, b0, packed, scales,
                                                                  zeros, Err);
         const int64_t rest = K - b0 - kBlock;
         if (rest > 0)
@@ -361,7 +382,7 @@ const char *shape_problem(int64_t K, int64_t N, int group) {
 }
 
 struct FullLayout {
-    size_t h, scratch, work, info, loop_at, total;
+    size_t h, scratch, info, loop_at, total;
     LoopLayout loop;
 };
 
@@ -369,8 +390,7 @@ FullLayout full_layout(int64_t K, int64_t N) {
     FullLayout F;
     F.h = 0;
     F.scratch = up256(sizeof(float) * size_t(K) * size_t(K));
-    F.work = up256(F.scratch + sizeof(float) * size_t(K) * size_t(K));
-    F.info = up256(F.work + solver_work_bytes(K));
+    F.info = up256(F.scratch + sizeof(float) * linalg_scratch_floats(K));
     F.loop_at = up256(F.info + 256);
     F.loop = loop_layout(K, N, F.loop_at);
     F.total = F.loop.total;
@@ -437,20 +457,16 @@ extern "C" int w4_gptq(const void *W, const void *X, int xt, int64_t Mc, int64_t
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     float *H = reinterpret_cast<float *>(ws + F.h);
-    // 1. H = 2 X^T X: column-major, the K x Mc matrix X (ld K) times its transpose
-    int st = w4::blas_gemm_f32("w4_gptq (Hessian)", false, true, static_cast<int>(K),
-                               static_cast<int>(K), static_cast<int>(Mc), 2.0f, X, xt,
-                               static_cast<int>(K), X, xt, static_cast<int>(K), 0.0f, H,
-                               static_cast<int>(K), s);
+    // 1. H = 2 X^T X (fp32 accumulation; the tiles on and above the diagonal)
+    int st = w4::hessian(X, xt, Mc, K, H, s);
     if (st != W4_OK) return st;
     // 2. damping
     w4::gptq_damp<<<1, 1024, 0, s>>>(H, K, percdamp);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return w4::cuda_fail("gptq_damp launch", e);
     // 3. U, the upper Cholesky factor of H^-1 (in place)
-    st = w4::solver_inverse_factor(fn, H, static_cast<int>(K), reinterpret_cast<float *>(ws + F.scratch),
-                                   ws + F.work, w4::solver_work_bytes(K),
-                                   reinterpret_cast<int *>(ws + F.info), s);
+    st = w4::inverse_factor(fn, H, K, reinterpret_cast<float *>(ws + F.scratch),
+                            reinterpret_cast<int *>(ws + F.info), s);
     if (st != W4_OK) return st;
     if (U_out) {
         e = cudaMemcpyAsync(U_out, H, sizeof(float) * size_t(K) * size_t(K), cudaMemcpyDeviceToDevice, s);

@@ -55,6 +55,11 @@ int launch_decode(const void *X, int xt, int64_t M, const uint8_t *packed, const
                   const float *zeros, int64_t K, int64_t N, void *Y, void *workspace,
                   size_t workspace_bytes, cudaStream_t stream);
 
+// M = 1, K % 512 == 0, K <= 4096: the CUDA-core GEMV; needs no workspace
+bool gemv1_supported(int64_t M, int64_t K);
+int launch_gemv1(const void *X, int xt, const uint8_t *packed, const float *scales,
+                 const float *zeros, int64_t K, int64_t N, void *Y, cudaStream_t stream);
+
 // decode path for M <= 8, K <= 4096 (warp-level tensor-core GEMV); needs no workspace
 bool gemv_supported(int64_t M, int64_t K);
 int launch_gemv(const void *X, int xt, int64_t M, const uint8_t *packed, const float *scales,
@@ -64,20 +69,23 @@ int launch_gemv(const void *X, int xt, int64_t M, const uint8_t *packed, const f
 int launch_prefill(const void *X, int xt, int64_t M, const uint8_t *packed, const float *scales,
                    const float *zeros, int64_t K, int64_t N, void *Y, cudaStream_t stream);
 
+// ---- GPTQ's dense linear algebra on the device (w4_linalg.cu) ----
+// H = 2 X^T X (fp32, [K][K] row-major; only the tiles on and above the
+// diagonal are written) from X [Mc][K] (W4_F16 / W4_BF16).
+int hessian(const void *X, int xt, int64_t Mc, int64_t K, float *H, cudaStream_t stream);
+// fp32 words of scratch inverse_factor needs for an n x n matrix.
+size_t linalg_scratch_floats(int64_t n);
+// In place: H (n x n fp32, the upper triangle read) -> U, the upper Cholesky
+// factor of H^-1 (row-major, zeros below the diagonal).  n % 64 == 0.
+// Synchronizes `stream` once to read the factorization status (info_dev: one
+// int of device memory); W4_ERR_INVALID_ARG if H is not positive definite.
+int inverse_factor(const char *fn, float *H, int64_t n, float *scratch, int *info_dev,
+                   cudaStream_t stream);
+
 // ---- NVIDIA libraries for plain dense linear algebra (w4_libs.cu) ----
 // C [m x n] fp32 (column-major, ldc) = alpha * op(A) op(B) + beta * C with
 // 16-bit A and B (types W4_F16 / W4_BF16), fp32 accumulation (cuBLAS GemmEx).
 int blas_gemm_f32(const char *fn, bool trans_a, bool trans_b, int m, int n, int k, float alpha,
                   const void *A, int at, int lda, const void *B, int bt, int ldb, float beta,
                   float *C, int ldc, cudaStream_t stream);
-// Work bytes reserved for solver_inverse_factor on an n x n matrix.
-size_t solver_work_bytes(int64_t n);
-// In place: H (n x n fp32, symmetric) -> the upper Cholesky factor U of H^-1
-// in row-major order (zeros below the diagonal); scratch is another n x n
-// fp32 buffer.  Synchronizes `stream` once to read the factorization statuses
-// (info_dev: 2 ints of device memory); W4_ERR_INVALID_ARG if H is not
-// positive definite.
-int solver_inverse_factor(const char *fn, float *H, int n, float *scratch, void *work,
-                          size_t work_bytes, int *info_dev, cudaStream_t stream);
-
 }  // namespace w4
