@@ -48,12 +48,12 @@ METRIC = "W4A16 g128 dequant-GEMM TB/s (decode) & TFLOPS (prefill) vs B200 roofl
 GROUP = 128
 
 # DRAM traffic of one decode launch (M=1, K=4096, N=12288: the dominant
-# kernel of the step, gemv_kernel of csrc/w4_gemv.cu) from one ncu capture
-# (dram__bytes_read.sum + dram__bytes_write.sum; profiles/gemv_kernel_m1_k4096_n12288.md),
+# kernel of the step, gemv1_kernel of csrc/w4_gemv1.cu) from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum; profiles/gemv1_kernel_m1_k4096_n12288.md),
 # valid only for the kernel source it was taken on: reported as null once
 # that source has changed.
-DECODE_SRC = "w4_gemv.cu"
-DECODE_TRAFFIC = {"bytes": None, "source_sha256_16": ""}
+DECODE_SRC = "w4_gemv1.cu"
+DECODE_TRAFFIC = {"bytes": 28366336, "source_sha256_16": "cd2f8a7ea77609c6"}
 
 
 # ---------------------------------------------------------------------------- helpers
@@ -327,7 +327,7 @@ def run_ours(args, ws_, rank, local):
     cur = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] if os.path.exists(src) else ""
     traffic = DECODE_TRAFFIC["bytes"] if (cur == DECODE_TRAFFIC["source_sha256_16"]
                                           and dom["N"] == 12288) else None
-    roof = {"bound": "hbm", "kernel": "gemv_kernel (w4a16_gemm, M=1)",
+    roof = {"bound": "hbm", "kernel": "gemv1_kernel (w4a16_gemm, M=1)",
             "achieved": round(dom["gbs"], 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": round(dom["gbs"] / pk["hbm_gbs"], 4), "traffic": traffic,
             "peak_source": pk["source"], "bytes_per_launch": dom["bytes"],
