@@ -55,7 +55,8 @@ typedef enum {
     W4_ERR_INVALID_ARG = 1, /* bad shape, null pointer, K % group != 0, ... */
     W4_ERR_UNSUPPORTED = 2, /* valid but not implemented (group size, alignment, dtype) */
     W4_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed while enqueueing */
-    W4_ERR_TIMEOUT = 4      /* a bounded device-side wait ran out (see w4_device_status) */
+    W4_ERR_TIMEOUT = 4,     /* a bounded device-side wait ran out (see w4_device_status) */
+    W4_ERR_BOUNDS = 5       /* an in-kernel bounds check of the W4_DEBUG build failed */
 } w4_status;
 
 typedef enum { W4_F16 = 0, W4_BF16 = 1 } w4_dtype;
@@ -100,8 +101,10 @@ int w4_quantize(const void *W, int wt, int64_t K, int64_t N, int group, int sym,
  * partials it reads, so one workspace serves any number of calls of any
  * shapes issued one after another on ONE stream.  Calls that may overlap on
  * the GPU (other streams) need separate workspaces.  A call whose bounded
- * wait ran out (w4_device_status reports W4_ERR_TIMEOUT) may stop partway and
- * leave counters armed: zero-fill the workspace again before reusing it.
+ * wait ran out, or (W4_DEBUG build) whose bounds check failed
+ * (w4_device_status reports W4_ERR_TIMEOUT or W4_ERR_BOUNDS), may stop
+ * partway and leave counters armed: zero-fill the workspace again before
+ * reusing it.
  */
 size_t w4a16_workspace_bytes(int64_t M, int64_t K, int64_t N, int group);
 
@@ -279,10 +282,33 @@ int w4_gptq_quantize(const void *W, int wt, int64_t K, int64_t N, int group, int
 
 /*
  * w4_device_status -- reads (and, if reset != 0, clears) the current device's
- * status word that kernels set when a bounded wait runs out.  Synchronizes the
- * device first.  Returns W4_OK, W4_ERR_TIMEOUT, or W4_ERR_CUDA if the read fails.
+ * status word that kernels set when a bounded wait runs out or, in the
+ * W4_DEBUG build, when a bounds check fails.  Synchronizes the device first.
+ * Returns W4_OK, W4_ERR_BOUNDS (a check failed; takes precedence),
+ * W4_ERR_TIMEOUT, or W4_ERR_CUDA if the read fails.
  */
 int w4_device_status(int reset);
+
+/*
+ * W4_DEBUG build (the pages have no counterpart; it stands in for a memory
+ * checker).  Built with -DW4_DEBUG (python -m weight_only_int4_pack_b200.build
+ * --debug, which writes libw4a16_debug.so), the decode, GEMV, prefill and
+ * quantizer kernels check every global and shared-memory index and every
+ * bulk / tensor copy they issue against the extents of their buffers.  A
+ * failed check does not trap: it sets the status word (W4_ERR_BOUNDS, read
+ * by w4_device_status) with the file and source line of the first failure,
+ * and the thread skips the access, so the context stays usable and the
+ * results of that call are undefined.  The normal build has no checks.
+ *
+ * w4_debug_build -- 1 if this library was built with W4_DEBUG, else 0.
+ * w4_debug_first_failure -- synchronizes the device and writes the file id
+ *   and line of the first failed check since the status word was last
+ *   cleared (0 and 0 if none); does not clear it.  File ids: 1 w4_quantize.cu,
+ *   2 w4_decode.cu, 3 w4_prefill.cu, 4 w4_gemv.cu, 5 w4_gemv1.cu.  Returns
+ *   W4_OK, W4_ERR_INVALID_ARG for a null pointer, or W4_ERR_CUDA.
+ */
+int w4_debug_build(void);
+int w4_debug_first_failure(int *file_id, int *line);
 
 /*
  * w4_selftest_wait_timeout -- failure-detection self-test (the pages have no
@@ -312,7 +338,7 @@ const char *w4_status_string(int status);
 /* ABI version of this header: (major << 16) | minor. */
 int w4_abi_version(void);
 
-#define W4A16_ABI_VERSION 0x00010002
+#define W4A16_ABI_VERSION 0x00010003
 
 #ifdef __cplusplus
 }

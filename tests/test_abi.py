@@ -80,12 +80,13 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert w4.w4_abi_version() == 0x00010002
+    assert w4.w4_abi_version() == 0x00010003
     assert w4.w4_status_string(0) == "W4_OK"
     assert w4.w4_status_string(1) == "W4_ERR_INVALID_ARG"
     assert w4.w4_status_string(2) == "W4_ERR_UNSUPPORTED"
     assert w4.w4_status_string(3) == "W4_ERR_CUDA"
     assert w4.w4_status_string(4) == "W4_ERR_TIMEOUT"
+    assert w4.w4_status_string(5) == "W4_ERR_BOUNDS"
     assert w4.w4_status_string(99) == "W4_ERR_UNKNOWN"
 
 

@@ -39,16 +39,20 @@ __all__ = [
     "w8a8_workspace_bytes", "w8a8_linear", "W8_INT8", "W8_E4M3", "W8_COL_NONE", "W8_COL_MUL",
     "W8_COL_DIV",
     "Workspace", "W4_OK", "W4_ERR_INVALID_ARG", "W4_ERR_UNSUPPORTED", "W4_ERR_CUDA",
-    "W4_ERR_TIMEOUT", "W4_F16", "W4_BF16",
+    "W4_ERR_TIMEOUT", "W4_ERR_BOUNDS", "W4_F16", "W4_BF16", "w4_debug_build",
+    "w4_debug_first_failure",
 ]
 
 W4_OK, W4_ERR_INVALID_ARG, W4_ERR_UNSUPPORTED, W4_ERR_CUDA, W4_ERR_TIMEOUT = 0, 1, 2, 3, 4
+W4_ERR_BOUNDS = 5
 W4_F16, W4_BF16 = 0, 1
 W8_INT8, W8_E4M3 = 0, 1
 W8_COL_NONE, W8_COL_MUL, W8_COL_DIV = 0, 1, 2
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-lib_path = os.path.join(_PKG, "lib", "libw4a16.so")
+# W4_DEBUG=1 in the environment selects the build with in-kernel bounds checks
+lib_path = os.path.join(_PKG, "lib", "libw4a16_debug.so" if os.environ.get("W4_DEBUG") == "1"
+                        else "libw4a16.so")
 _lib = None
 
 
@@ -89,6 +93,10 @@ def load() -> ctypes.CDLL:
     lib.w4a16_gemm_noalloc.restype = I
     lib.w4_selftest_wait_timeout.argtypes = [ctypes.c_uint, P]
     lib.w4_selftest_wait_timeout.restype = I
+    lib.w4_debug_build.argtypes = []
+    lib.w4_debug_build.restype = I
+    lib.w4_debug_first_failure.argtypes = [ctypes.POINTER(I), ctypes.POINTER(I)]
+    lib.w4_debug_first_failure.restype = I
     lib.w4_awq_search_workspace_bytes.argtypes = [I64, I64, I64, I]
     lib.w4_awq_search_workspace_bytes.restype = SZ
     lib.w4_awq_search.argtypes = [P, P, I, I64, I64, I64, I, I, P, I, P, P, P, P, P, P, P, SZ, P]
@@ -177,13 +185,29 @@ _ws_epoch = [0]
 
 
 def w4_device_status(reset: bool = True) -> int:
-    """Status word set by kernels whose bounded waits ran out (synchronizes).
-    On W4_ERR_TIMEOUT every Workspace of this module is zero-filled again
-    before its next use, as include/w4a16.h asks."""
+    """Status word set by kernels whose bounded waits ran out, or whose
+    W4_DEBUG bounds checks failed (synchronizes).  On W4_ERR_TIMEOUT or
+    W4_ERR_BOUNDS every Workspace of this module is zero-filled again before
+    its next use, as include/w4a16.h asks."""
     st = int(load().w4_device_status(int(bool(reset))))
-    if st == W4_ERR_TIMEOUT:
+    if st in (W4_ERR_TIMEOUT, W4_ERR_BOUNDS):
         _ws_epoch[0] += 1
     return st
+
+
+def w4_debug_build() -> bool:
+    """True if the loaded library was built with W4_DEBUG (in-kernel bounds checks)."""
+    return bool(load().w4_debug_build())
+
+
+def w4_debug_first_failure() -> tuple[int, int]:
+    """(file id, source line) of the first failed W4_DEBUG check since the
+    status word was last cleared; (0, 0) if none.  Synchronizes; does not clear."""
+    f, ln = ctypes.c_int(0), ctypes.c_int(0)
+    st = int(load().w4_debug_first_failure(ctypes.byref(f), ctypes.byref(ln)))
+    if st != W4_OK:
+        raise W4Error("w4_debug_first_failure", st)
+    return f.value, ln.value
 
 
 def w4_selftest_wait_timeout(timeout_us: int = 1000, stream=None) -> None:

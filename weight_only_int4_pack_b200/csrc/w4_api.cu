@@ -218,6 +218,7 @@ const char *w4_status_string(int status) {
         case W4_ERR_UNSUPPORTED: return "W4_ERR_UNSUPPORTED";
         case W4_ERR_CUDA: return "W4_ERR_CUDA";
         case W4_ERR_TIMEOUT: return "W4_ERR_TIMEOUT";
+        case W4_ERR_BOUNDS: return "W4_ERR_BOUNDS";
         default: return "W4_ERR_UNKNOWN";
     }
 }
@@ -265,7 +266,28 @@ int w4_device_status(int reset) {
         if ((e = cudaMemcpyToSymbol(g_w4_status, &zero, sizeof zero)) != cudaSuccess)
             return w4::cuda_fail("clear status word", e);
     }
+    if (v & 2u) return W4_ERR_BOUNDS;
     return v ? W4_ERR_TIMEOUT : W4_OK;
+}
+
+int w4_debug_build(void) {
+#ifdef W4_DEBUG
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+int w4_debug_first_failure(int *file_id, int *line) {
+    if (!file_id || !line) return w4::set_error(W4_ERR_INVALID_ARG, "w4_debug_first_failure", "null pointer");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return w4::cuda_fail("cudaDeviceSynchronize", e);
+    unsigned v = 0;
+    if ((e = cudaMemcpyFromSymbol(&v, g_w4_status, sizeof v)) != cudaSuccess)
+        return w4::cuda_fail("read status word", e);
+    *file_id = static_cast<int>((v >> 2) & 63u);
+    *line = static_cast<int>(v >> 8);
+    return W4_OK;
 }
 
 }  // extern "C"

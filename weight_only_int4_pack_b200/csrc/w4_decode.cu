@@ -47,10 +47,13 @@
 #include <cuda_fp16.h>
 #include <stdio.h>
 
+#include "w4_debug.cuh"
 #include "w4_internal.cuh"
 
 namespace w4 {
 namespace {
+
+[[maybe_unused]] constexpr unsigned kDbgFile = 2;  // W4_DEBUG file id
 
 constexpr int kGroup = 128;
 constexpr int kUnitRows = 128;                      // weight rows per unit (= TMEM lanes)
@@ -396,6 +399,7 @@ struct Shared {
     uint32_t tmem_base;
     int abort_flag;
 };
+static_assert(sizeof(Shared) <= 512, "the exchange buffer starts 512 bytes after the barriers");
 
 // Warp roles (10 warps): 0 producer, 1 TMEM allocator + MMA issuer,
 // 2..9 dequant (warp w: TMEM lane quarter w % 4, the units of parity
@@ -428,6 +432,17 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
     const int u1 = range_start(wk, c + 1);
     const int nu = u1 - u0;
     const int G = wk.G;
+    // W4_DEBUG: [p, p + bytes) inside the stage ring, itself inside this
+    // launch's shared memory; a TMA box start with a 16-byte aligned x
+    [[maybe_unused]] auto ring_ok = [&](const void *p, uint32_t bytes) {
+        return in_range(smem_u32(p), bytes, smem_u32(ring), uint64_t(S) * C::kBytes) &&
+               in_range(smem_u32(ring), uint64_t(S) * C::kBytes + 512 + 4 * NN * 32 * 4,
+                        smem_u32(smem_raw), dyn_smem_bytes());
+    };
+    [[maybe_unused]] auto wbox_ok = [&](int x, int y) {
+        return x >= 0 && x % 16 == 0 && x < K / 2 && y >= 0 && y < N;
+    };
+    [[maybe_unused]] auto xbox_ok = [&](int x) { return x >= 0 && x % 8 == 0; };
 
     // The packed weights are inputs no earlier kernel writes: thread 0 (the
     // producer's TMA lane) requests the codes of the CTA's first two units as
@@ -453,6 +468,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         int rb = u0 / wk.KS, ks = u0 - (u0 / wk.KS) * wk.KS;
         for (int it = 0; it < early; ++it) {
             const uint32_t fb = smem_u32(&sh->full[it]);
+            if (!W4_CHECK(ring_ok(ring + it * C::kBytes, C::kBytes) &&
+                              wbox_ok(ks * (kUnitK / 2), rb * kUnitRows),
+                          status))
+                break;
             mbar_arrive_tx(fb, C::kTmaBytes);
             tma_load_2d(smem_u32(ring + it * C::kBytes), &tmap_w, ks * (kUnitK / 2), rb * kUnitRows,
                         fb);
@@ -488,6 +507,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                 for (int q = 0; q < 4; ++q) {
                     const int r = lane + 32 * q;
                     const int64_t n = min(rb * kUnitRows + r, N - 1);
+                    if (!W4_CHECK(n >= 0 && g0 >= 0 && g1 < G && ring_ok(zz + 2 * r, 8), status)) continue;
                     cp_async4(smem_u32(zz + 2 * r), zeros + n * G + g0);
                     cp_async4(smem_u32(zz + 2 * r + 1), zeros + n * G + g1);
                 }
@@ -497,10 +517,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
         auto issue_x = [&](int ks, uint8_t *st, uint32_t fb) {
 #pragma unroll
             for (int b = 0; b < 4; ++b)
-                tma_load_2d(smem_u32(st + kUnitBytes + b * C::kXBox), &tmap_x, ks * kUnitK + 64 * b, 0,
+                if (W4_CHECK(xbox_ok(ks * kUnitK + 64 * b) && ring_ok(st + kUnitBytes + b * C::kXBox, C::kXBox),
+                             status))
+                    tma_load_2d(smem_u32(st + kUnitBytes + b * C::kXBox), &tmap_x, ks * kUnitK + 64 * b, 0,
                             fb);
         };
         auto issue_w = [&](int rb, int ks, uint8_t *st, uint32_t fb) {
+            if (!W4_CHECK(ring_ok(st, C::kBytes) && wbox_ok(ks * (kUnitK / 2), rb * kUnitRows), status))
+                return;
             mbar_arrive_tx(fb, C::kTmaBytes);
             tma_load_2d(smem_u32(st), &tmap_w, ks * (kUnitK / 2), rb * kUnitRows, fb);
         };
@@ -651,6 +675,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             float *xb = xbuf + q * NN * 32 + lane;
             const uint32_t par = nflush & 1;
             ++nflush;
+            if (!W4_CHECK_WARP(in_range(smem_u32(xb), 4, smem_u32(ring) + uint64_t(S) * C::kBytes + 512,
+                                        4 * NN * 32 * 4) &&
+                                   in_range(smem_u32(xb + 32 * (NN - 1)), 4,
+                                            smem_u32(ring) + uint64_t(S) * C::kBytes + 512, 4 * NN * 32 * 4),
+                               status))
+                return false;
             if (p == 1) {
                 if (!warp_wait(smem_u32(&sh->xfree[q]), par ^ 1, abort_flag, status)) return false;
 #pragma unroll
@@ -666,7 +696,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
             if (lane == 0) mbar_arrive(smem_u32(&sh->xfree[q]));
             const int n = rb * kUnitRows + r;
             if (rb * wk.KS >= u0 && (rb + 1) * wk.KS <= u1) {  // whole row block in this range
-                if (n < N) {
+                if (n < N && W4_CHECK(n >= 0 && M <= NN, status)) {
 #pragma unroll
                     for (int m = 0; m < NN; ++m)
                         if (m < M) store_out<XT>(Y, (int64_t)m * N + n, acc[m]);
@@ -674,6 +704,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                 return true;
             }
             const int slot = 2 * c + (rb == u0 / wk.KS ? 0 : 1);
+            if (!W4_CHECK_WARP(partial != nullptr && slot >= 0 && slot < 2 * wk.P && M <= NN &&
+                                   rb >= 0 && rb * 8 + q < static_cast<int>(kCounterBytes / sizeof(unsigned)),
+                               status))
+                return false;
             float *dst = partial + ((int64_t)slot * kUnitRows + r) * M;
 #pragma unroll
             for (int m = 0; m < NN; ++m)
@@ -730,6 +764,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                 if (fold) {
                     // scales of the folded unit (row r), from global memory
                     const int64_t n = min(frb * kUnitRows + r, N - 1);
+                    if (!W4_CHECK_WARP(n >= 0 && fks >= 0 && 2 * fks < G, status)) {
+                        ok = false;
+                        break;
+                    }
                     const float *sp = scales + n * G + 2 * fks;
                     s0 = __ldg(sp);
                     s1 = 2 * fks + 1 < G ? __ldg(sp + 1) : 0.0f;
@@ -740,6 +778,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                         break;
                     }
                     const uint8_t *st = ring + s * C::kBytes;
+                    if (!W4_CHECK_WARP(ring_ok(st, C::kBytes) && r * 128 + 128 <= kUnitBytes &&
+                                           ring_ok(st + C::kZOff + 8 * r, 8),
+                                       status)) {
+                        ok = false;
+                        break;
+                    }
                     const float *zz = reinterpret_cast<const float *>(st + C::kZOff) + 2 * r;
                     zero_bias<XT>(zeros ? zz[0] : 8.0f, zb0, zq0);
                     zero_bias<XT>(zeros ? zz[1] : 8.0f, zb1, zq1);
@@ -825,7 +869,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant_
                 if (prev != (unsigned)(cl - cf)) continue;
                 __syncwarp();
                 const int n = prb * kUnitRows + r;
-                if (n < N) {
+                if (n < N && W4_CHECK(n >= 0 && cf >= 0 && cl < wk.P, status)) {
                     for (int m = 0; m < M; ++m) {
                         float v = 0.0f;
                         for (int cc = cf; cc <= cl; ++cc) {

@@ -45,17 +45,23 @@
 //     only after it (weights -- codes, scales, zero points -- before).
 //
 // The kernel has no unbounded wait: cp.async groups complete on their own,
-// and the only barriers are CTA-wide bar.sync that every warp reaches.
+// the CTA-wide bar.sync are reached by every warp, and the one spin (a warp
+// kSlots tiles ahead waiting for a reduction slot) is bounded: when it runs
+// out it sets the library's status word (W4_ERR_TIMEOUT).  The W4_DEBUG build
+// checks every global and shared-memory index and copy (w4_debug.cuh).
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include "w4_debug.cuh"
 #include "w4_half.cuh"
 #include "w4_internal.cuh"
 #include "w4_tc.cuh"
 
 namespace w4 {
 namespace {
+
+[[maybe_unused]] constexpr unsigned kDbgFile = 4;  // W4_DEBUG file id
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
@@ -215,7 +221,7 @@ template <int XT>
 __global__ void __launch_bounds__(kThreads, 2)
     gemv_kernel(const uint8_t *__restrict__ packed, const float *__restrict__ scales,
                 const float *__restrict__ zeros, const uint16_t *__restrict__ X,
-                uint16_t *__restrict__ Y, int M, int K, int N) {
+                uint16_t *__restrict__ Y, int M, int K, int N, unsigned *status) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
@@ -254,6 +260,13 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int ra = r0 + i * kTile + gq;
             const bool oka = ra < r1, okb = ra + 8 < r1;
             const uint8_t *qa = pa + i * tile_bytes, *qb = qa + 8 * static_cast<int64_t>(kb);
+            if (!W4_CHECK(ra >= 0 && (!oka || ra < N) && (!okb || ra + 8 < N) && gA + ng <= G &&
+                              in_range(st, kStageBytes, sb, dyn_smem_bytes()) &&
+                              in_range(st, kStageBytes, sb + L.ring, L.x - L.ring),
+                          status)) {
+                cp_async_commit();
+                return;
+            }
 #pragma unroll
             for (int gi = 0; gi < kGPW; ++gi) {
                 if (gi < ng) {
@@ -293,9 +306,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int e = threadIdx.x; e < M * KC; e += kThreads) {
         const int m = e / KC, kc = e - m * KC;
         const int g = kc >> 4, tt = (kc >> 2) & 3, w4 = kc & 3;
+        const uint32_t a = sb + L.x + m * L.XS + g * 256 + tt * 64 + ((w4 ^ (tt >> 1)) << 4);
+        if (!W4_CHECK(m < M && kc < KC && in_range(a, 16, sb + L.x, L.tab - L.x), status)) continue;
         const uint4 v = __ldg(reinterpret_cast<const uint4 *>(X + static_cast<int64_t>(m) * K) + kc);
-        sts128(sb + L.x + m * L.XS + g * 256 + tt * 64 + ((w4 ^ (tt >> 1)) << 4),
-               make_uint4(v.x, v.z, v.y, v.w));
+        sts128(a, make_uint4(v.x, v.z, v.y, v.w));
     }
     cta_sync();
     // entries (g, m), m < M, one thread each, from the shared copy of x (the
@@ -312,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             widen8<XT>(v, f);  // words stored as (k,k+1), (k+4,k+5), (k+2,k+3), (k+6,k+7)
             acc += ((f[0] + f[1]) + (f[4] + f[5])) + ((f[2] + f[3]) + (f[6] + f[7]));
         }
-        tab[g * 8 + m] = XT == W4_F16 ? acc * 0x1p-24f : acc;
+        if (W4_CHECK(g < G && m < 8, status)) tab[g * 8 + m] = XT == W4_F16 ? acc * 0x1p-24f : acc;
     }
     for (int e = threadIdx.x; e < G * 8; e += kThreads)
         if ((e & 7) >= M) tab[e] = 0.f;
@@ -345,6 +359,19 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int gi = 0; gi < kGPW; ++gi) {
             if (gi < ng) {
+                const uint32_t ss = st + sza - t * kTile * 4 + gi * kTile * 4 - gq * 4;
+                // the lane's code reads, its x reads (pieces xoff[0..3] = [0, 64)
+                // of its slice), its scale and zero-point reads; one vote for
+                // the warp, whose MMAs below are warp-collective
+                if (!W4_CHECK_WARP(in_range(st + gi * (kTile * 64) + ca, 16, st, kStageCodes) &&
+                                       in_range(st + gi * (kTile * 64) + cb, 16, st, kStageCodes) &&
+                                       in_range(xrow + (gA + gi) * 256, 64, sb + L.x, L.tab - L.x) &&
+                                       in_range(ss + gq * 4, 4, st + kStageCodes, kGPW * kTile * 4) &&
+                                       in_range(ss + (gq + 8) * 4, 4, st + kStageCodes, kGPW * kTile * 4) &&
+                                       in_range(ss + kGPW * kTile * 4 + (gq + 8) * 4, 4,
+                                                st + kStageCodes + kGPW * kTile * 4, kGPW * kTile * 4),
+                                   status))
+                    continue;
                 const uint4 c0 = lds128(st + gi * (kTile * 64) + ca);
                 const uint4 c1 = lds128(st + gi * (kTile * 64) + cb);
                 // activation pairs of the 4 slice words, stored per 16-byte
@@ -361,7 +388,6 @@ __global__ void __launch_bounds__(kThreads, 2)
                 for (int j = 0; j < 4; ++j)
                     step<XT>(dA, dB, cw0[j], cw1[j], xv[j].x, xv[j].y, xv[j].z, xv[j].w);
                 // fold: y[r][n] += s_r * (sum x u - z_r sum x)
-                const uint32_t ss = st + sza - t * kTile * 4 + gi * kTile * 4 - gq * 4;
                 const float s0 = lds32f(ss + gq * 4), s1 = lds32f(ss + (gq + 8) * 4);
                 float z0 = 8.f, z1 = 8.f;
                 if (asym) {
@@ -399,10 +425,16 @@ __global__ void __launch_bounds__(kThreads, 2)
         const unsigned want = static_cast<unsigned>(i / kSlots);
         if (*gen != want) {  // a warp kSlots tiles ahead of the slowest one
             const unsigned long long t0 = tc::globaltimer();
-            while (*gen != want && tc::globaltimer() - t0 < tc::kWaitNs) {
+            while (*gen != want) {
+                if (tc::globaltimer() - t0 > tc::kWaitNs) {
+                    if (lane == 0) atomicOr(status, 1u);
+                    break;
+                }
             }
         }
         const uint32_t sl = sb + L.red + slot * (kWarps * 32 * 16);
+        if (!W4_CHECK_WARP(in_range(sl + (warp * 32 + lane) * 16, 16, sb + L.red, L.sync - L.red), status))
+            continue;
         sts128(sl + (warp * 32 + lane) * 16, make_uint4(__float_as_uint(y[0]), __float_as_uint(y[1]),
                                                         __float_as_uint(y[2]), __float_as_uint(y[3])));
         __syncwarp();
@@ -426,11 +458,11 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int row0 = r0 + i * kTile;
             const int ra = row0 + gq, rbw = row0 + gq + 8;
             const int m0 = 2 * t, m1 = 2 * t + 1;
-            if (ra < r1) {
+            if (ra < r1 && W4_CHECK(ra >= 0 && ra < N, status)) {
                 if (m0 < M) Y[static_cast<int64_t>(m0) * N + ra] = narrow1<XT>(a[0]);
                 if (m1 < M) Y[static_cast<int64_t>(m1) * N + ra] = narrow1<XT>(a[1]);
             }
-            if (rbw < r1) {
+            if (rbw < r1 && W4_CHECK(rbw >= 0 && rbw < N, status)) {
                 if (m0 < M) Y[static_cast<int64_t>(m0) * N + rbw] = narrow1<XT>(a[2]);
                 if (m1 < M) Y[static_cast<int64_t>(m1) * N + rbw] = narrow1<XT>(a[3]);
             }
@@ -461,6 +493,8 @@ int launch_t(const uint8_t *packed, const float *scales, const float *zeros, con
         if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(gemv smem)", e);
         attr_done[dev] = true;
     }
+    unsigned *status = device_status_ptr();
+    if (!status) return W4_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads);
@@ -473,7 +507,7 @@ int launch_t(const uint8_t *packed, const float *scales, const float *zeros, con
     cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, packed, scales, zeros,
                                        static_cast<const uint16_t *>(X), static_cast<uint16_t *>(Y),
-                                       M, K, N);
+                                       M, K, N, status);
     if (e != cudaSuccess) return cuda_fail("cudaLaunchKernelEx(gemv)", e);
     return W4_OK;
 }

@@ -39,17 +39,21 @@
 //
 // Every mbarrier wait is bounded; a wait that runs out sets the library's
 // status word (W4_ERR_TIMEOUT), the warp stops, and it waits (bounded) for its
-// copies in flight before it exits.
+// copies in flight before it exits.  The W4_DEBUG build checks every global
+// and shared-memory index and every copy against its buffer (w4_debug.cuh).
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include "w4_debug.cuh"
 #include "w4_half.cuh"
 #include "w4_internal.cuh"
 #include "w4_tc.cuh"
 
 namespace w4 {
 namespace {
+
+[[maybe_unused]] constexpr unsigned kDbgFile = 5;  // W4_DEBUG file id
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
@@ -221,6 +225,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t r = row_of(j);
         const uint32_t st = sstage + d * sbytes;
         const uint32_t bar = sbar + d * 8;
+        if (!W4_CHECK(r >= 0 && r < N && d >= 0 && d < kStages &&
+                          in_range(st, sbytes, sx, dyn_smem_bytes()) &&
+                          in_range(bar, 8, sx, dyn_smem_bytes()),
+                      status))
+            return;
         tc::mbar_arrive_tx(bar, sbytes);
         bulk_g2s(st, packed + r * cbytes, cbytes, bar);
         bulk_g2s(st + cbytes, scales + r * G, gbytes, bar);
@@ -245,8 +254,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // reading piece p of slices i..i+7 hit 8 different bank quads.
     for (int t = threadIdx.x; t < K / 8; t += kThreads) {
         const int i = t >> 2, p = t & 3;
+        const uint32_t a = sx + i * 64 + ((p ^ ((i >> 1) & 3)) << 4);
+        if (!W4_CHECK(t >= 0 && in_range(a, 16, sx, static_cast<uint64_t>(K) * 2), status)) continue;
         const uint4 v = __ldg(reinterpret_cast<const uint4 *>(X) + t);
-        sts128(sx + i * 64 + ((p ^ ((i >> 1) & 3)) << 4), v);
+        sts128(a, v);
     }
     __syncthreads();
 
@@ -261,7 +272,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         float s = 0.f, tb = 0.f;
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
-            xr[q][p] = on ? lds128(sx + ic * 64 + ((p ^ ((ic >> 1) & 3)) << 4)) : make_uint4(0, 0, 0, 0);
+            const uint32_t a = sx + ic * 64 + ((p ^ ((ic >> 1) & 3)) << 4);
+            xr[q][p] = on && W4_CHECK(in_range(a, 16, sx, static_cast<uint64_t>(K) * 2), status)
+                           ? lds128(a)
+                           : make_uint4(0, 0, 0, 0);
             float f[8];
             widen8<XT>(xr[q][p], f);
             // fp16: k = 8p + {0,1,4,5} carry offset 1024, k = 8p + {2,3,6,7}
@@ -304,6 +318,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int q = 0; q < C; ++q) {
                     const int i = lane + 32 * q;
                     const int ic = i < KW ? i : KW - 1;
+                    if (!W4_CHECK(in_range(st + ic * 16, 16, st, cbytes) &&
+                                      in_range(st + cbytes + (ic >> 2) * 4, 4, st + cbytes, gbytes) &&
+                                      (!asym || in_range(st + cbytes + gbytes + (ic >> 2) * 4, 4,
+                                                         st + cbytes + gbytes, gbytes)) &&
+                                      in_range(st, sbytes, sx, dyn_smem_bytes()),
+                                  status))
+                        continue;  // per-lane work only: no collective until reduce4
                     const uint4 cw = lds128(st + ic * 16);
                     const float sc = lds32f(st + cbytes + (ic >> 2) * 4);
                     const float zc = asym ? lds32f(st + cbytes + gbytes + (ic >> 2) * 4) : 8.f;
@@ -324,7 +345,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float r = reduce4(part, lane);
         const int t = (lane >> 3) & 3;
-        if ((lane & 7) == 0 && jb + t < nrows) Y[row_of(jb + t)] = narrow1<XT>(r);
+        if ((lane & 7) == 0 && jb + t < nrows &&
+            W4_CHECK(row_of(jb + t) >= 0 && row_of(jb + t) < N, status))
+            Y[row_of(jb + t)] = narrow1<XT>(r);
     }
 }
 

@@ -53,11 +53,14 @@
 #include <stdio.h>
 
 
+#include "w4_debug.cuh"
 #include "w4_internal.cuh"
 #include "w4_tc.cuh"
 
 namespace w4 {
 namespace {
+
+[[maybe_unused]] constexpr unsigned kDbgFile = 3;  // W4_DEBUG file id
 
 constexpr int kBM = 128;       // weight rows per tile (MMA M)
 constexpr int kBN = 256;       // activation rows per tile (MMA N)
@@ -170,6 +173,7 @@ struct Smem {
     uint32_t tmem_base;
     int abort_flag;
 };
+static_assert(sizeof(Smem) <= 256, "the barrier area of kSmemBytes");
 
 // Dequantizes the two stages of group g of the current tile (stage counter
 // base `it`) for this thread's A-tile row dr: waits for the codes, writes the
@@ -180,6 +184,7 @@ __device__ __forceinline__ bool dequant_group(int g, uint32_t it, int n_d, int G
                                               const float *__restrict__ zeros, const uint8_t *cs,
                                               uint8_t *as, int dr, Smem *sm,
                                               volatile int *abort_flag, unsigned *status) {
+    if (!W4_CHECK_WARP(n_d >= 0 && g >= 0 && g < G, status)) return false;
     const float z = zeros ? __ldg(zeros + (int64_t)n_d * G + g) : 8.0f;
     uint32_t zb, zq;
     zero_bias<XT>(z, zb, zq);
@@ -192,6 +197,11 @@ __device__ __forceinline__ bool dequant_group(int g, uint32_t it, int n_d, int G
         if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm->full[s]), ph, abort_flag, status)))
             return false;
         const uint8_t *crow = cs + s * kCodeTileBytes + dr * (kBK / 2);
+        if (!W4_CHECK_WARP(in_range(smem_u32(crow), kBK / 2, smem_u32(cs), uint64_t(kStages) * kCodeTileBytes) &&
+                               in_range(smem_u32(as + s * kATileBytes + dr * 128), 128, smem_u32(as),
+                                        uint64_t(kStages) * kATileBytes),
+                           status))
+            return false;
         const uint4 w0 = *reinterpret_cast<const uint4 *>(crow);
         const uint4 w1 = *reinterpret_cast<const uint4 *>(crow + 16);
         uint8_t *arow = as + s * kATileBytes + dr * 128;
@@ -273,6 +283,16 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
                         break;
                     }
                     const uint32_t fb = smem_u32(&sm->full[s]);
+                    // W4_DEBUG: 16-byte aligned box starts inside the tensors, and the
+                    // stage ring (then the barriers) inside this launch's shared memory
+                    if (!W4_CHECK((ks * kBK) % 8 == 0 && ks * kBK < K && mt * kBN < M &&
+                                      (ks * (kBK / 2)) % 16 == 0 && nt * kBM < N &&
+                                      in_range(smem_u32(sm), sizeof(Smem), smem_u32(smem_raw),
+                                               dyn_smem_bytes()),
+                                  status)) {
+                        ok = false;
+                        break;
+                    }
                     mbar_arrive_tx(fb, kXTileBytes + kCodeTileBytes);
                     tma_load_2d(smem_u32(xs + s * kXTileBytes), &tmap_x, ks * kBK, mt * kBN, fb);
                     tma_load_2d(smem_u32(cs + s * kCodeTileBytes), &tmap_w, ks * (kBK / 2),
@@ -366,6 +386,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             const int nt = tile % n_tiles, mt = tile / n_tiles;
             const int n_e = nt * kBM + er;
             const int n_ec = min(n_e, N - 1);
+            if (!W4_CHECK_WARP(n_ec >= 0 && G >= 1, status)) break;
 #pragma unroll
             for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
             float s_next = __ldg(scales + (int64_t)n_ec * G + 0);
@@ -400,7 +421,7 @@ prefill_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
             }
             if (!ok) break;
             // store this thread's row n_e for its 128 columns m
-            if (n_e < N) {
+            if (n_e < N && W4_CHECK(n_e >= 0 && mt * kBN < M, status)) {
                 const int m0 = mt * kBN + colhalf * 128;
 #pragma unroll
                 for (int i = 0; i < 128; ++i) {

@@ -28,10 +28,13 @@
 #include <cuda_fp16.h>
 #include <float.h>
 
+#include "w4_debug.cuh"
 #include "w4_internal.cuh"
 
 namespace w4 {
 namespace {
+
+[[maybe_unused]] constexpr unsigned kDbgFile = 1;  // W4_DEBUG file id
 
 constexpr int kThreads = 128;
 constexpr int kPer = 16;                // consecutive k per thread
@@ -172,7 +175,7 @@ __global__ void __launch_bounds__(kThreads)
 quantize_kernel(const uint16_t *__restrict__ W, int64_t K, int64_t N,
                 const float *__restrict__ col_scale, uint32_t *__restrict__ packed,
                 float *__restrict__ scales, float *__restrict__ zeros, int64_t tiles_k,
-                int64_t tiles) {
+                int64_t tiles, unsigned *status) {
     constexpr int LPG = GROUP / kPer;  // lanes per group (2, 4, 8 or 16)
     const int t = threadIdx.x;
     const int lane = t & 31;
@@ -187,7 +190,7 @@ quantize_kernel(const uint16_t *__restrict__ W, int64_t K, int64_t N,
         if (FOLD) {
 #pragma unroll
             for (int j = 0; j < kPer; ++j) cs[j] = 1.0f;
-            if (valid_k) {
+            if (valid_k && W4_CHECK(k >= 0 && k + kPer <= K, status)) {
 #pragma unroll
                 for (int v = 0; v < kPer / 4; ++v) {
                     const float4 c = __ldg(reinterpret_cast<const float4 *>(col_scale + k) + v);
@@ -203,7 +206,8 @@ quantize_kernel(const uint16_t *__restrict__ W, int64_t K, int64_t N,
             for (int i = 0; i < kRowUnroll; ++i) {
                 const int64_t row = row0 + rr + i;
                 raw[i][0] = raw[i][1] = make_uint4(0, 0, 0, 0);
-                if (valid_k && row < N) {
+                if (valid_k && row < N &&
+                    W4_CHECK(row >= 0 && k >= 0 && k + kPer <= K && (k & 7) == 0, status)) {
                     const uint4 *src = reinterpret_cast<const uint4 *>(W + row * K + k);
                     raw[i][0] = __ldcs(src);
                     raw[i][1] = __ldcs(src + 1);
@@ -262,13 +266,17 @@ quantize_kernel(const uint16_t *__restrict__ W, int64_t K, int64_t N,
                     if (near0 || !fast_ok) codes_exact<SYM>(w, s, zp, bits);
                     if (near1 || !fast_ok) codes_exact<SYM>(w + 8, s, zp, bits + 8);
                 }
-                if (valid_k) {
+                if (valid_k &&
+                    W4_CHECK(row >= 0 && row < N && k >= 0 && k + kPer <= K && ((row * K + k) & 15) == 0,
+                             status)) {
                     reinterpret_cast<uint2 *>(packed)[(row * K + k) >> 4] =
                         make_uint2(pack8(bits), pack8(bits + 8));
                     if ((lane % LPG) == 0) {
                         const int64_t gi = row * G + k / GROUP;
-                        scales[gi] = s;
-                        zeros[gi] = zp;
+                        if (W4_CHECK(gi >= 0 && gi < N * G, status)) {
+                            scales[gi] = s;
+                            zeros[gi] = zp;
+                        }
                     }
                 }
             }
@@ -294,9 +302,11 @@ int launch_t(const void *W, int64_t K, int64_t N, const float *col_scale, uint8_
     const int64_t tiles = tiles_k * ((N + kRowsPerTile - 1) / kRowsPerTile);
     int64_t grid = static_cast<int64_t>(di.sm_count) * blocks_per_sm;
     if (grid > tiles) grid = tiles;
+    unsigned *status = device_status_ptr();
+    if (!status) return W4_ERR_CUDA;
     kern<<<static_cast<unsigned>(grid), kThreads, 0, stream>>>(
         static_cast<const uint16_t *>(W), K, N, col_scale, reinterpret_cast<uint32_t *>(packed),
-        scales, zeros, tiles_k, tiles);
+        scales, zeros, tiles_k, tiles, status);
     return cuda_status(cudaGetLastError());
 }
 
