@@ -113,9 +113,43 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
+// Encoded tensor maps are cached per host thread, direct-mapped by a hash of
+// everything the encoding depends on (the map holds only the address, the
+// extents, the stride, the box and the modes), so a layer called again with
+// the same buffers skips the driver call.  A buffer freed and another
+// allocated at the same address with the same extents gets the same map,
+// which is exactly the map it needs.
+struct MapKey {
+    const void *ptr;
+    uint64_t inner, outer, row_bytes;
+    uint32_t box_inner, box_outer;
+    int dt, swz;
+    bool operator==(const MapKey &o) const {
+        return ptr == o.ptr && inner == o.inner && outer == o.outer && row_bytes == o.row_bytes &&
+               box_inner == o.box_inner && box_outer == o.box_outer && dt == o.dt && swz == o.swz;
+    }
+};
+struct MapEntry {
+    CUtensorMap map;
+    MapKey key;
+    bool valid;
+};
+constexpr int kMapCache = 64;
+thread_local MapEntry t_maps[kMapCache];
+
 int make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *ptr, uint64_t inner,
                 uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
                 CUtensorMapSwizzle swz, const char *what) {
+    const MapKey key = {ptr, inner, outer, row_bytes, box_inner, box_outer, (int)dt, (int)swz};
+    uint64_t h = reinterpret_cast<uintptr_t>(ptr) >> 8;
+    h = h * 0x9E3779B97F4A7C15ull ^ inner ^ (outer << 20) ^ (row_bytes << 7) ^
+        (uint64_t(box_inner) << 40) ^ (uint64_t(box_outer) << 48) ^ (uint64_t(dt) << 56) ^
+        (uint64_t(swz) << 60);
+    MapEntry &slot = t_maps[(h ^ (h >> 29)) % kMapCache];
+    if (slot.valid && slot.key == key) {
+        *map = slot.map;
+        return W4_OK;
+    }
     auto fn = tensor_map_encoder();
     if (!fn) return W4_ERR_CUDA;
     cuuint64_t dims[2] = {inner, outer};
@@ -130,6 +164,9 @@ int make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *ptr, uint6
         snprintf(buf, sizeof buf, "cuTensorMapEncodeTiled returned CUresult %d", (int)r);
         return set_error(W4_ERR_CUDA, what, buf);
     }
+    slot.map = *map;
+    slot.key = key;
+    slot.valid = true;
     return W4_OK;
 }
 
