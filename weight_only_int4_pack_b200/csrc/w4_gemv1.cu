@@ -9,8 +9,11 @@
 // of codes per weight and does one multiply-add per weight, so it is bound by
 // HBM, not by any arithmetic pipe; the kernel is shaped for that:
 //
-//   * No split-K, no workspace.  Each CTA owns an equal contiguous range of
-//     weight rows; its warps take the rows round robin.  A row's codes, scales
+//   * No split-K, no workspace.  Three CTAs of four warps per SM (so that a
+//     CTA of the next launch in the stream can be resident, and start its
+//     weight copies, while this launch's last CTAs finish); each CTA owns an
+//     equal contiguous range of weight rows and its warps take the rows
+//     round robin.  A row's codes, scales
 //     and zero points are contiguous in HBM and come in with three 1-D bulk
 //     copies (cp.async.bulk) into a per-warp ring of shared-memory stages, so
 //     every warp has four rows in flight without holding them in registers,
@@ -55,12 +58,13 @@ namespace {
 
 [[maybe_unused]] constexpr unsigned kDbgFile = 5;  // W4_DEBUG file id
 
-constexpr int kWarps = 8;
+constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr int kStages = 4;      // rows in flight per warp
 constexpr int kBatch = 4;       // rows reduced together
 constexpr int kMaxK = 4096;     // x slices held in registers: K / 64 words per lane
 constexpr int kGroup = 128;
+constexpr int kCtasPerSm = 3;  // 12 warps per SM; a CTA of the next launch can join early
 
 static_assert(kBatch == kStages, "a batch uses every stage once");
 
@@ -193,7 +197,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, unsigne
 
 // C = 32-k slices per lane = ceil(K / 1024).
 template <int XT, int C>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
     gemv1_kernel(const uint8_t *__restrict__ packed, const float *__restrict__ scales,
                 const float *__restrict__ zeros, const uint16_t *__restrict__ X,
                 uint16_t *__restrict__ Y, int K, int N, unsigned *status) {
@@ -400,7 +404,8 @@ int launch_gemv1(const void *X, int xt, const uint8_t *packed, const float *scal
     if (st != W4_OK) return st;
     if (di.cc_major != 10) return set_error(W4_ERR_UNSUPPORTED, "w4a16_gemm", "needs an sm_100 GPU");
     const int k = static_cast<int>(K), n = static_cast<int>(N);
-    const int grid = static_cast<int>(N < di.sm_count ? N : di.sm_count);
+    const int64_t most = static_cast<int64_t>(kCtasPerSm) * di.sm_count;
+    const int grid = static_cast<int>(N < most ? N : most);
     const size_t smem = static_cast<size_t>(k) * 2 +
                         static_cast<size_t>(kWarps) * kStages * (stage_bytes_for(k, zeros != nullptr) + 8);
     const int C = (k + 1023) / 1024;
