@@ -54,10 +54,13 @@ def test_every_m(M, dtype):
 
 
 @pytest.mark.parametrize("M", [1, 2])
-@pytest.mark.parametrize("N", [1, 2, 7, 15, 16, 17, 147, 148, 149, 296, 2371, 4101])
+@pytest.mark.parametrize("N", [1, 2, 7, 15, 16, 17, 147, 148, 149, 296, 443, 444, 445, 889, 1777, 2371,
+                               4101])
 def test_row_counts(N, M):
-    """Rows per CTA from 0 to many, partial batches of 4 rows (M = 1) and
-    partial tiles of 16 rows (M = 2)."""
+    """Rows per CTA from 1 to many (the M = 1 GEMV runs up to three CTAs per
+    SM: N around 444 and its multiples gives CTAs of 1 to 5 rows and warps
+    with none), partial batches of 4 rows (M = 1) and partial tiles of 16
+    rows (M = 2)."""
     run(M, N, 4096, False, "f16", N + M)
 
 
