@@ -16,6 +16,7 @@ wrong columns or group parameters taken from the original weights fails one.
 """
 import numpy as np
 import pytest
+import scipy.linalg
 import torch
 
 import oracle
@@ -38,6 +39,25 @@ def test_hessian_and_factor():
     assert np.allclose(np.tril(U, -1), 0.0)
     Hd = H + 0.01 * np.mean(np.diag(H)) * np.eye(128)
     np.testing.assert_allclose(U.T @ U @ Hd, np.eye(128), atol=1e-8)
+
+
+@pytest.mark.parametrize("K,Mc,seed", [(128, 48, 2), (256, 512, 3), (384, 200, 4)])
+def test_reversed_cholesky_gives_the_same_factor(K, Mc, seed):
+    """The route the library's device code takes to U, checked in fp64 with
+    numpy's and scipy's own routines: with P the index reversal and L the lower Cholesky
+    factor of P (H + lambda I) P, P L^-1 P is upper triangular with a positive
+    diagonal and (P L^-1 P)^T (P L^-1 P) = (H + lambda I)^-1, so by the
+    uniqueness of the Cholesky factor it is the oracle's U."""
+    X = synth.activations(Mc, K, seed, salient_frac=0.02)
+    H = oracle.gptq_hessian(bits(X), oracle.F16)
+    Hd = H + 0.01 * np.mean(np.diag(H)) * np.eye(K)
+    P = np.eye(K)[::-1]
+    L = np.linalg.cholesky(P @ Hd @ P)
+    Ur = P @ scipy.linalg.solve_triangular(L, np.eye(K), lower=True) @ P
+    assert np.allclose(np.tril(Ur, -1), 0.0, atol=0.0)
+    assert (np.diag(Ur) > 0).all()
+    U = oracle.gptq_inverse_factor(H, 0.01)
+    np.testing.assert_allclose(Ur, U, rtol=0, atol=1e-9 * np.abs(U).max())
 
 
 @pytest.mark.parametrize("sym", [True, False])
