@@ -54,8 +54,11 @@ def calib_error(packed, scales, zeros, W, X, K, sym):
 
 
 @pytest.mark.parametrize("sym", [False, True])
-@pytest.mark.parametrize("N,K,Mc", [(64, 256, 512), (300, 512, 1024), (96, 512, 256)])
+@pytest.mark.parametrize("N,K,Mc", [(64, 256, 512), (300, 512, 1024), (96, 512, 256),
+                                    (40, 384, 256), (24, 640, 300)])
 def test_whole_pipeline(N, K, Mc, sym):
+    """K = 384 and 640 (6 and 10 diagonal blocks of 64) run the triangular
+    inverse's partial last pair and its unpaired last block."""
     W, X = layer(N, K, Mc, "f16", 7 + N + K)
     p, s, z, U = w4.w4_gptq(W.to(DEV), X.to(DEV), sym=sym, return_u=True)
     torch.cuda.synchronize()
