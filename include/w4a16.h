@@ -230,7 +230,7 @@ int w4_awq_search(const void *W, const void *X, int xt, int64_t Mc, int64_t K, i
 /*
  * w4_gptq_workspace_bytes / w4_gptq_quantize_workspace_bytes -- device
  * scratch bytes of w4_gptq and w4_gptq_quantize (0 for a shape they reject):
- * about 8 K^2 + 4 N K + 512 N bytes (w4_gptq) and 4 N K + 512 N (the loop).
+ * about 9 K^2 + 4 N K + 512 N bytes (w4_gptq) and 4 N K + 512 N (the loop).
  */
 size_t w4_gptq_workspace_bytes(int64_t Mc, int64_t K, int64_t N, int group);
 size_t w4_gptq_quantize_workspace_bytes(int64_t K, int64_t N, int group);
