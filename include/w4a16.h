@@ -120,8 +120,9 @@ size_t w4a16_workspace_bytes(int64_t M, int64_t K, int64_t N, int group);
  *   fp32 (the integer (u - zero) is exact in the 16-bit operand type; the
  *   group scale multiplies the fp32 partial sum of its group) and rounded
  *   once to the output dtype.
- *   M = 1 with K % 512 == 0 and K <= 4096 runs the CUDA-core GEMV (one CTA
- *   per SM, whole rows streamed per warp, no workspace); other 1 <= M <= 8
+ *   M = 1 with K % 512 == 0 and K <= 4096 runs the CUDA-core GEMV (three
+ *   CTAs of four warps per SM, whole rows streamed per warp, no workspace);
+ *   other 1 <= M <= 8
  *   with K <= 4096 the small-M GEMV on warp-level tensor-core MMAs (whole
  *   rows, no workspace); other M <= 32 the persistent stream-K decode path
  *   on tcgen05; larger M runs the

@@ -7,7 +7,9 @@
 // (zhiyuanblog.org/blog/llm-quantization) §2.2-§2.3.  At small M the layer is
 // bound by streaming the packed weights from HBM, so the kernel is built to
 // keep HBM busy from the first cycle to the last and to spend as few issue
-// slots per weight as possible:
+// slots per weight as possible.  (launch_decode, at the end, sends M = 1
+// with K <= 4096 to the CUDA-core GEMV of w4_gemv1.cu and other M <= 8 with
+// K <= 4096 to the warp-MMA GEMV of w4_gemv.cu; this kernel serves the rest.)
 //
 //   * Persistent, one CTA per SM.  The packed matrix is cut into units of
 //     128 weight rows x 256 k (16 KB of codes, two groups).  The units, in
